@@ -1,0 +1,215 @@
+/*
+ * fluxbin.h -- C-ABI of the B200 (sm_100a) FluxBin LUT GEMV library, libfluxbin.so.
+ *
+ * FluxBin ("FluxBin: Flexible LUT-based Ultra-low-bit LLM Inference by
+ * Algorithm-Kernel Synergy") stores a weight matrix W (M rows = output
+ * features, N columns = input features) as
+ *
+ *     W = sum_{k < Kb} diag(r_k) B_k diag(c_k)                       (global branch)
+ *       + salient refinement on a column set S, |S| = n_sal:
+ *         sum_{s < Ks} diag(rs_s) Bs_s diag(cs_s), column t of Bs_s being column S[t] of W
+ *
+ * with B_k, Bs_s in {-1,+1} (summary, Section 3 "Quantization" and "Salient-
+ * Aware Hybrid Bases").  The library evaluates y = W x for a batch of fp16
+ * activations without ever forming a floating-point W: for every sub-vector
+ * of mu activation columns it builds a table of the 2^mu signed partial sums
+ * of c (.) x (scale fusion, Section 3 "LUT-Based GEMV Kernel", Appendix C.1),
+ * streams the packed sign bits from HBM, uses each mu-bit pattern as a table
+ * index, accumulates in fp32 and applies the row scale after accumulation.
+ * The salient branch runs through the same kernel on its dense M x n_sal
+ * sign matrix, its activations and scales gathered through S at run time
+ * (Section 3 "Virtual Columnar Mapping").
+ *
+ * Conventions for every entry point:
+ *   - Return value: FLUXBIN_OK (0) or a negative fluxbin_status.  No call
+ *     throws, aborts or prints.  Arguments are validated before any CUDA call,
+ *     so an argument error leaves the device and the stream untouched.
+ *   - fp16 values travel as uint16_t bit patterns (IEEE binary16).
+ *   - Pointers named d_* are device pointers, owned by the caller, never freed
+ *     or retained after the call returns; no call allocates device memory.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default
+ *     stream).  Device calls are asynchronous on that stream: they launch and
+ *     return without synchronising.
+ *   - Only one GPU architecture is built: sm_100a (B200).  Launch failures
+ *     are reported as FLUXBIN_ERR_CUDA.
+ *
+ * ---------------------------------------------------------------------------
+ * Packed sign layout (the device layout; a pure index function)
+ * ---------------------------------------------------------------------------
+ * One branch (the global one: nb = Kb bases over ncols = N columns; the
+ * salient one: nb = Ks bases over ncols = n_sal dense columns) with
+ * sub-vector length mu in {4, 8} and nb in {1, 2, 4} is stored as follows.
+ *
+ *   P  = 32 / nb            sub-vectors of one base in a unit
+ *   U  = ceil(ncols / (P*mu)) units: column blocks of P*mu columns
+ *   Ms = ceil(M / 32)       row slabs of 32 rows
+ *   words: Ms * U chunks, chunk (s, u) at word offset (s*U + u) * 32*mu,
+ *          each chunk 32*mu uint32 words (1 KiB for mu = 8, 512 B for mu = 4).
+ *
+ * The sign of base k at row i and column n (n < ncols) is one bit, set for
+ * +1 and clear for -1; every padding bit (rows >= M, columns >= ncols) is 0:
+ *   s = i / 32, L = i % 32                      row slab and lane
+ *   jg = n / mu, t = n % mu                     sub-vector and bit within it
+ *   u = jg / P, j = jg % P                      unit and sub-vector within it
+ *   a = (k - L/P) mod nb                        (mod taken in 0..nb-1)
+ *   q = a*P + ((j - L) mod P)                   step at which lane L visits it
+ *   pos  = q*mu + t
+ *   word = (s*U + u)*32*mu + ((pos / 128)*32 + L)*4 + (pos / 32) % 4
+ *   bit  = pos % 32
+ *
+ * Reading: lane L of a warp owns row 32*s + L.  Over its 32 steps q it visits
+ * the unit's 32 (base, sub-vector) tables in the order
+ *   base k = (q/P + L/P) mod nb, sub-vector j = (L + q) mod P,
+ * so at every step the 32 lanes read 32 different tables.  Table (k, j) lives
+ * in shared-memory bank k*P + j; no two lanes ever hit the same bank.  The
+ * 32*mu bits a lane consumes for one unit are contiguous (mu/4 128-bit words,
+ * interleaved across the warp's lanes so that every warp load is one
+ * contiguous 512-byte line).
+ *
+ * ---------------------------------------------------------------------------
+ * Scale layouts (fp16)
+ * ---------------------------------------------------------------------------
+ *   c  [Kb][N], cs [Ks][n_sal]                  column scales
+ *   r  [Kb][M]            (row_scale_group == 0: one per row)
+ *   r  [Kb][ceil(N/G)][M] (row_scale_group == G > 0: one per row per G-column
+ *                          block, Appendix C.2 "block-wise row scales")
+ *   rs [Ks][M] or [Ks][ceil(n_sal/Gs)][M]       (sal_scale_group == Gs)
+ *   x  [B][N], y [B][M] (row-major; y fp16 or fp32)
+ *   idx[n_sal] int32, strictly increasing, < N  (the salient column set S)
+ */
+#ifndef FLUXBIN_H
+#define FLUXBIN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum fluxbin_status {
+    FLUXBIN_OK = 0,
+    FLUXBIN_ERR_INVALID_ARG = -1,  /* null pointer where data is needed, bad flag */
+    FLUXBIN_ERR_BAD_SHAPE = -2,    /* negative or inconsistent sizes, bad salient index list */
+    FLUXBIN_ERR_MISALIGNED = -3,   /* a device pointer lacks the alignment stated below */
+    FLUXBIN_ERR_UNSUPPORTED = -4,  /* mu not in {4,8}; Kb not in {1,2,4}; Ks not in {0,1,2,4};
+                                      B > 16; a scale block that does not hold whole units */
+    FLUXBIN_ERR_SMEM_BUDGET = -5,  /* the tables for this shape do not fit in shared memory */
+    FLUXBIN_ERR_WORKSPACE = -6,    /* workspace missing or smaller than fluxbin_workspace_bytes() */
+    FLUXBIN_ERR_CUDA = -7          /* a CUDA runtime call or the kernel launch failed */
+} fluxbin_status;
+
+/* Plain-old-data description of one layer. */
+typedef struct fluxbin_layer_desc {
+    int32_t M;                /* output features (rows of W), >= 0 */
+    int32_t N;                /* input features (columns of W), >= 0 */
+    int32_t Kb;               /* global bases: 1, 2 or 4 */
+    int32_t Ks;               /* salient bases: 0 (no salient branch), 1, 2 or 4 */
+    int32_t n_sal;            /* salient columns, 0 <= n_sal <= N (0 when Ks == 0) */
+    int32_t mu;               /* LUT sub-vector length: 4 or 8 */
+    int32_t row_scale_group;  /* 0: one row scale per row; G > 0: one per row per G columns */
+    int32_t sal_scale_group;  /* 0: one salient row scale per row; Gs > 0: one per Gs salient columns */
+} fluxbin_layer_desc;
+
+/* Flags for the device entry points. */
+#define FLUXBIN_FLAG_ACCUMULATE   1u  /* y += W x (else y = W x) */
+#define FLUXBIN_FLAG_Y_FP32       2u  /* y is float32 (else fp16, round to nearest even) */
+#define FLUXBIN_FLAG_EARLY_WEIGHTS 4u /* programmatic dependent launch: start streaming this
+                                         layer's packed signs before the preceding kernel on the
+                                         stream has finished.  The caller promises that no kernel
+                                         still running before this call writes the layer's packed
+                                         words.  x, y, scales and workspace are always read only
+                                         after the preceding kernel has completed. */
+
+/* Human-readable name of a status code (static storage, never NULL). */
+const char* fluxbin_status_string(int status);
+
+/* Library version: major*10000 + minor*100 + patch. */
+int fluxbin_version(void);
+
+/*
+ * Sizes of the packed sign arrays of a layer, in bytes (words_bytes for the
+ * global branch, swords_bytes for the salient branch; 0 when it is absent).
+ * Follows the packed sign layout above.  Host only; no CUDA call.
+ * Errors: INVALID_ARG (null desc or outputs), BAD_SHAPE, UNSUPPORTED.
+ */
+int fluxbin_packed_sizes(const fluxbin_layer_desc* desc, size_t* words_bytes, size_t* swords_bytes);
+
+/*
+ * Host packer: the binary bases as sign bits in uint32 words, streamed later
+ * without ever being turned back into floats (summary, Section 3 "LUT-Based
+ * GEMV Kernel"; news article: weights "streamed in a compressed Uint32
+ * format").  It also validates the salient column list S that Virtual
+ * Columnar Mapping gathers through (Section 3 "Virtual Columnar Mapping").
+ *
+ *   signs     host int8 [Kb][M][N], each +1 or -1
+ *   sal_signs host int8 [Ks][M][n_sal], each +1 or -1 (NULL when Ks == 0 or n_sal == 0)
+ *   sal_idx   host int32 [n_sal], strictly increasing, each in [0, N)
+ *   words_out  host, caller-allocated, fluxbin_packed_sizes().words_bytes bytes
+ *   swords_out host, caller-allocated, swords_bytes bytes (NULL when absent)
+ * Every output word is written (padding bits 0).  Host only; no CUDA call.
+ * Errors: INVALID_ARG (null arrays), BAD_SHAPE (a sign not +-1, S not strictly
+ * increasing or out of range), UNSUPPORTED.  On error the outputs are unspecified.
+ */
+int fluxbin_pack(const fluxbin_layer_desc* desc, const int8_t* signs, const int8_t* sal_signs,
+                 const int32_t* sal_idx, uint32_t* words_out, uint32_t* swords_out);
+
+/*
+ * Device workspace needed by fluxbin_linear / fluxbin_lut_gemv for a layer of
+ * M rows at batch B: split-K partial sums (fp32 [B][ceil(M/32)*32]) and one
+ * arrival counter per row group and batch chunk.  Host only.
+ * The workspace must be zero-filled once before its first use (for example
+ * with cudaMemsetAsync); every call leaves it zero-filled again.  Calls that
+ * may run concurrently on the GPU must not share a workspace.
+ * Errors: INVALID_ARG (null output), BAD_SHAPE (M < 0 or B < 0).
+ */
+int fluxbin_workspace_bytes(int32_t M, int32_t B, size_t* bytes);
+
+/*
+ * One dense branch (the kernel that Virtual Columnar Mapping reuses):
+ *   y[b][i] (+)= sum_k r_k(i) * sum_{n < ncols} B_k[i][n] c_k[n] x[b][col(n)]
+ * with col(n) = d_gather[n] (or n when d_gather is NULL).
+ *   M, N         rows of W and the length of every x row
+ *   ncols, nbases, mu   geometry of the packed branch (nbases in {1,2,4})
+ *   row_scale_group     0 (d_r is [nbases][M]) or G (d_r is [nbases][ceil(ncols/G)][M]);
+ *                       G must be a multiple of the unit width (32/nbases)*mu
+ *   d_words      packed signs, 16-byte aligned (layout above)
+ *   d_r, d_c     fp16 scales; d_c is [nbases][ncols]
+ *   d_gather     int32 [ncols] or NULL.  An entry outside [0, N) contributes 0.
+ *   d_x          fp16 [B][N];  B in [0, 16]
+ *   d_y          [B][M], fp16 or fp32 per FLUXBIN_FLAG_Y_FP32; 4-byte aligned for fp32
+ *   flags        FLUXBIN_FLAG_*
+ *   d_workspace, workspace_bytes   see fluxbin_workspace_bytes (may be NULL/0 only
+ *                when that function reports fewer bytes than given)
+ * M == 0 or B == 0 returns FLUXBIN_OK without launching.
+ * Errors: INVALID_ARG, BAD_SHAPE, MISALIGNED, UNSUPPORTED, SMEM_BUDGET, WORKSPACE, CUDA.
+ */
+int fluxbin_lut_gemv(int32_t M, int32_t N, int32_t ncols, int32_t nbases, int32_t mu,
+                     int32_t row_scale_group,
+                     const uint32_t* d_words, const uint16_t* d_r, const uint16_t* d_c,
+                     const int32_t* d_gather, const uint16_t* d_x, int32_t B,
+                     void* d_y, uint32_t flags, void* d_workspace, size_t workspace_bytes,
+                     void* stream);
+
+/*
+ * The full layer, global and salient branches in one launch:
+ *   y[b] (+)= W x[b]   (W as at the top of this file)
+ *   d_words  [global packed signs], d_r, d_c   global scales
+ *   d_swords [salient packed signs], d_rs, d_cs, d_idx (S)   salient branch
+ *            (all four ignored when Ks == 0 or n_sal == 0)
+ * Other arguments as for fluxbin_lut_gemv.  Graph-capturable: no allocation,
+ * no synchronisation, no host-device copy.
+ * Errors: INVALID_ARG, BAD_SHAPE, MISALIGNED, UNSUPPORTED, SMEM_BUDGET, WORKSPACE, CUDA.
+ */
+int fluxbin_linear(const fluxbin_layer_desc* desc,
+                   const uint32_t* d_words, const uint16_t* d_r, const uint16_t* d_c,
+                   const uint32_t* d_swords, const uint16_t* d_rs, const uint16_t* d_cs,
+                   const int32_t* d_idx, const uint16_t* d_x, int32_t B,
+                   void* d_y, uint32_t flags, void* d_workspace, size_t workspace_bytes,
+                   void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FLUXBIN_H */

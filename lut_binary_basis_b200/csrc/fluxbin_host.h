@@ -1,0 +1,44 @@
+// Host-side validation shared by the packer and the device entry points.
+#pragma once
+
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/fluxbin.h"
+#include "fluxbin_layout.h"
+
+namespace fluxbin {
+
+inline bool valid_nb(int nb) { return nb == 1 || nb == 2 || nb == 4; }
+inline bool valid_mu(int mu) { return mu == 4 || mu == 8; }
+
+inline bool has_salient(const fluxbin_layer_desc& d) { return d.Ks > 0 && d.n_sal > 0; }
+
+// Checks the shape fields of a layer description.
+inline int validate_desc(const fluxbin_layer_desc* d) {
+    if (!d) return FLUXBIN_ERR_INVALID_ARG;
+    if (d->M < 0 || d->N < 0 || d->n_sal < 0 || d->row_scale_group < 0 || d->sal_scale_group < 0)
+        return FLUXBIN_ERR_BAD_SHAPE;
+    if (!valid_mu(d->mu) || !valid_nb(d->Kb)) return FLUXBIN_ERR_UNSUPPORTED;
+    if (d->Ks != 0 && !valid_nb(d->Ks)) return FLUXBIN_ERR_UNSUPPORTED;
+    if (d->n_sal > d->N) return FLUXBIN_ERR_BAD_SHAPE;
+    if (d->Ks == 0 && d->n_sal != 0) return FLUXBIN_ERR_BAD_SHAPE;
+    // block-wise row scales: a block must hold whole units, so that the scale
+    // is constant across the unit a CTA accumulates before applying it
+    if (d->row_scale_group > 0 && d->row_scale_group % unit_cols(d->Kb, d->mu)) return FLUXBIN_ERR_UNSUPPORTED;
+    if (has_salient(*d) && d->sal_scale_group > 0 && d->sal_scale_group % unit_cols(d->Ks, d->mu))
+        return FLUXBIN_ERR_UNSUPPORTED;
+    return FLUXBIN_OK;
+}
+
+inline size_t workspace_bytes_for(int64_t M, int64_t B) {
+    if (M <= 0 || B <= 0) return 0;
+    const int64_t Mp = row_slabs(M) * kLanes;
+    const int64_t n_rg = (row_slabs(M) + kSlabsPerCta - 1) / kSlabsPerCta;
+    size_t acc = (size_t)(B * Mp) * sizeof(float);
+    acc = (acc + 255) & ~(size_t)255;
+    size_t cnt = (size_t)(n_rg * B) * sizeof(unsigned int);
+    return acc + ((cnt + 255) & ~(size_t)255);
+}
+
+}  // namespace fluxbin

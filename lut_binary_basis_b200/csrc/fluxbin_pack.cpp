@@ -1,0 +1,111 @@
+// Host packer and host-only queries of libfluxbin (no CUDA calls).
+//
+// The packer writes the +-1 bases as sign bits in uint32 words in the
+// device layout defined in include/fluxbin.h ("Packed sign layout"): the
+// FluxBin summary's Section 3 "LUT-Based GEMV Kernel" reads compressed
+// weights with bitwise operations, and the news article on FluxBin notes the
+// weights are streamed as compressed uint32 words, never rebuilt as floats.
+#include <string.h>
+
+#include "fluxbin_host.h"
+
+using namespace fluxbin;
+
+namespace {
+
+// Packs one branch: signs [nb][M][ncols] (+-1) -> words (device layout).
+int pack_branch(const int8_t* signs, int64_t M, int64_t ncols, int nb, int mu, uint32_t* words) {
+    const int P = subvecs_per_unit(nb);
+    const int64_t U = branch_units(ncols, nb, mu);
+    const int64_t total = branch_words(M, ncols, nb, mu);
+    memset(words, 0, (size_t)total * sizeof(uint32_t));
+    const int64_t nsub = (ncols + mu - 1) / mu;
+    for (int k = 0; k < nb; ++k) {
+        for (int64_t i = 0; i < M; ++i) {
+            const int8_t* row = signs + ((int64_t)k * M + i) * ncols;
+            const int64_t s = i / kLanes;
+            const int L = (int)(i % kLanes);
+            for (int64_t jg = 0; jg < nsub; ++jg) {
+                uint32_t pat = 0;
+                const int64_t n0 = jg * mu;
+                for (int t = 0; t < mu && n0 + t < ncols; ++t) {
+                    const int8_t v = row[n0 + t];
+                    if (v == 1) pat |= 1u << t;
+                    else if (v != -1) return FLUXBIN_ERR_BAD_SHAPE;
+                }
+                if (!pat) continue;
+                const int64_t u = jg / P;
+                const int j = (int)(jg % P);
+                const int q = visit_step(L, k, j, nb);
+                const int pos = q * mu;
+                const int64_t w = (s * U + u) * chunk_words(mu) + ((int64_t)(pos / 128) * kLanes + L) * 4 + (pos / 32) % 4;
+                words[w] |= pat << (pos % 32);
+            }
+        }
+    }
+    return FLUXBIN_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* fluxbin_status_string(int status) {
+    switch (status) {
+        case FLUXBIN_OK: return "ok";
+        case FLUXBIN_ERR_INVALID_ARG: return "invalid argument";
+        case FLUXBIN_ERR_BAD_SHAPE: return "bad shape";
+        case FLUXBIN_ERR_MISALIGNED: return "misaligned pointer";
+        case FLUXBIN_ERR_UNSUPPORTED: return "unsupported configuration";
+        case FLUXBIN_ERR_SMEM_BUDGET: return "shared-memory budget exceeded";
+        case FLUXBIN_ERR_WORKSPACE: return "workspace missing or too small";
+        case FLUXBIN_ERR_CUDA: return "CUDA error";
+        default: return "unknown status";
+    }
+}
+
+int fluxbin_version(void) { return 1 * 10000 + 0 * 100 + 0; }
+
+int fluxbin_packed_sizes(const fluxbin_layer_desc* desc, size_t* words_bytes, size_t* swords_bytes) {
+    if (!words_bytes || !swords_bytes) return FLUXBIN_ERR_INVALID_ARG;
+    const int st = validate_desc(desc);
+    if (st != FLUXBIN_OK) return st;
+    *words_bytes = (size_t)branch_words(desc->M, desc->N, desc->Kb, desc->mu) * sizeof(uint32_t);
+    *swords_bytes = has_salient(*desc)
+        ? (size_t)branch_words(desc->M, desc->n_sal, desc->Ks, desc->mu) * sizeof(uint32_t) : 0;
+    return FLUXBIN_OK;
+}
+
+int fluxbin_pack(const fluxbin_layer_desc* desc, const int8_t* signs, const int8_t* sal_signs,
+                 const int32_t* sal_idx, uint32_t* words_out, uint32_t* swords_out) {
+    const int st = validate_desc(desc);
+    if (st != FLUXBIN_OK) return st;
+    const fluxbin_layer_desc& d = *desc;
+    const int64_t nw = branch_words(d.M, d.N, d.Kb, d.mu);
+    if (nw > 0 && (!signs || !words_out)) return FLUXBIN_ERR_INVALID_ARG;
+    if (has_salient(d)) {
+        if (!sal_signs || !sal_idx || !swords_out) return FLUXBIN_ERR_INVALID_ARG;
+        for (int32_t t = 0; t < d.n_sal; ++t) {
+            if (sal_idx[t] < 0 || sal_idx[t] >= d.N) return FLUXBIN_ERR_BAD_SHAPE;
+            if (t > 0 && sal_idx[t] <= sal_idx[t - 1]) return FLUXBIN_ERR_BAD_SHAPE;
+        }
+    }
+    if (nw > 0) {
+        const int r = pack_branch(signs, d.M, d.N, d.Kb, d.mu, words_out);
+        if (r != FLUXBIN_OK) return r;
+    }
+    if (has_salient(d) && branch_words(d.M, d.n_sal, d.Ks, d.mu) > 0) {
+        const int r = pack_branch(sal_signs, d.M, d.n_sal, d.Ks, d.mu, swords_out);
+        if (r != FLUXBIN_OK) return r;
+    }
+    return FLUXBIN_OK;
+}
+
+int fluxbin_workspace_bytes(int32_t M, int32_t B, size_t* bytes) {
+    if (!bytes) return FLUXBIN_ERR_INVALID_ARG;
+    if (M < 0 || B < 0) return FLUXBIN_ERR_BAD_SHAPE;
+    *bytes = workspace_bytes_for(M, B);
+    return FLUXBIN_OK;
+}
+
+}  // extern "C"
