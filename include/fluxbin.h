@@ -96,7 +96,8 @@ typedef enum fluxbin_status {
                                       B > 16; a scale block that does not hold whole units */
     FLUXBIN_ERR_SMEM_BUDGET = -5,  /* the tables for this shape do not fit in shared memory */
     FLUXBIN_ERR_WORKSPACE = -6,    /* workspace missing or smaller than fluxbin_workspace_bytes() */
-    FLUXBIN_ERR_CUDA = -7          /* a CUDA runtime call or the kernel launch failed */
+    FLUXBIN_ERR_CUDA = -7,         /* a CUDA runtime call or the kernel launch failed */
+    FLUXBIN_ERR_SCRATCH_LIMIT = -8 /* the layer needs more scratch than FLUXBIN_STATIC_SCRATCH_BYTES */
 } fluxbin_status;
 
 /* Plain-old-data description of one layer. */
@@ -207,6 +208,42 @@ int fluxbin_linear(const fluxbin_layer_desc* desc,
                    const int32_t* d_idx, const uint16_t* d_x, int32_t B,
                    void* d_y, uint32_t flags, void* d_workspace, size_t workspace_bytes,
                    void* stream);
+
+/*
+ * fluxbin_linear for callers that cannot allocate device memory.  (An
+ * addition of this library; the FluxBin pages have no counterpart.)
+ *
+ * Some callers have no way to obtain a workspace: a plugin loaded into a host
+ * program that owns every byte of device memory through its own pool and
+ * forbids direct cudaMalloc, or a latency-critical loop that must never call
+ * cudaMalloc / cudaFree because those calls synchronise the device.  This
+ * entry point needs no workspace argument: its split-K scratch is a fixed
+ * array of FLUXBIN_STATIC_SCRATCH_BYTES in the library's own device memory,
+ * which every GPU that loads the library holds until the process exits.
+ *
+ *   - Same arguments and results as fluxbin_linear, without d_workspace and
+ *     workspace_bytes.  Nothing is allocated: no cudaMalloc, cudaFree or
+ *     allocating library routine is called.
+ *   - The first call on each device looks up the scratch address for that
+ *     device (with the device current); make that first call before any
+ *     stream capture begins.
+ *   - Each call first clears, on `stream`, the part of the scratch that must
+ *     start at zero (fluxbin_workspace_bytes(M, B) bytes), then launches.
+ *   - Every call on a device shares the one scratch array: calls that may
+ *     overlap on the GPU (different streams without ordering between them)
+ *     race and give wrong results.  Order them on one stream.
+ *   - A layer whose scratch need fluxbin_workspace_bytes(M, B) exceeds
+ *     FLUXBIN_STATIC_SCRATCH_BYTES is rejected with FLUXBIN_ERR_SCRATCH_LIMIT
+ *     before anything is launched (4 MiB covers, for example, M = 32768 at B = 16).
+ * Errors: as fluxbin_linear, plus SCRATCH_LIMIT; CUDA when the scratch address
+ * cannot be obtained or cleared.
+ */
+#define FLUXBIN_STATIC_SCRATCH_BYTES (4u << 20)
+int fluxbin_linear_static_scratch(const fluxbin_layer_desc* desc,
+                                  const uint32_t* d_words, const uint16_t* d_r, const uint16_t* d_c,
+                                  const uint32_t* d_swords, const uint16_t* d_rs, const uint16_t* d_cs,
+                                  const int32_t* d_idx, const uint16_t* d_x, int32_t B,
+                                  void* d_y, uint32_t flags, void* stream);
 
 #ifdef __cplusplus
 }

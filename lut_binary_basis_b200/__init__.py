@@ -8,6 +8,6 @@ it has not been built.
 """
 from . import synth  # noqa: F401
 from .fluxbin import (FLAG_ACCUMULATE, FLAG_EARLY_WEIGHTS, FLAG_Y_FP32, DeviceLayer, FluxbinError,  # noqa: F401
-                      FluxbinLibraryMissing, LayerDesc, fluxbin_linear, fluxbin_lut_gemv, fluxbin_pack,
-                      fluxbin_packed_sizes, fluxbin_status_string, fluxbin_version, fluxbin_workspace_bytes,
+                      FluxbinLibraryMissing, LayerDesc, fluxbin_linear, fluxbin_linear_static_scratch,
+                      fluxbin_lut_gemv, fluxbin_pack, fluxbin_packed_sizes, fluxbin_status_string, fluxbin_version, fluxbin_workspace_bytes,
                       new_workspace)

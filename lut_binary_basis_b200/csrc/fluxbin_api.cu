@@ -185,3 +185,65 @@ int fluxbin_linear(const fluxbin_layer_desc* desc, const uint32_t* d_words, cons
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Entry point without a workspace argument, for callers that cannot allocate
+// device memory (see fluxbin_linear_static_scratch in include/fluxbin.h).
+// ---------------------------------------------------------------------------
+
+// The scratch lives in the library's own device memory, one copy per device
+// that loads the library.  In host code this name is only a stand-in for the
+// symbol, not a device address: the address is looked up per device below.
+static __device__ __align__(256) unsigned char g_fluxbin_static_scratch[FLUXBIN_STATIC_SCRATCH_BYTES];
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+std::mutex g_scratch_mu;
+void* g_scratch_addr[kMaxDevices] = {};
+
+// Device address of the static scratch on the current device, looked up once
+// per device (with that device current) and cached.
+int static_scratch_address(void** out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return FLUXBIN_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_scratch_mu);
+    if (!g_scratch_addr[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_fluxbin_static_scratch) != cudaSuccess || !p) {
+            (void)cudaGetLastError();
+            return FLUXBIN_ERR_CUDA;
+        }
+        g_scratch_addr[dev] = p;
+    }
+    *out = g_scratch_addr[dev];
+    return FLUXBIN_OK;
+}
+
+}  // namespace
+
+extern "C" int fluxbin_linear_static_scratch(const fluxbin_layer_desc* desc, const uint32_t* d_words,
+                                             const uint16_t* d_r, const uint16_t* d_c, const uint32_t* d_swords,
+                                             const uint16_t* d_rs, const uint16_t* d_cs, const int32_t* d_idx,
+                                             const uint16_t* d_x, int32_t B, void* d_y, uint32_t flags,
+                                             void* stream) {
+    const int st = validate_desc(desc);
+    if (st != FLUXBIN_OK) return st;
+    if (B < 0) return FLUXBIN_ERR_BAD_SHAPE;
+    if (B > kMaxBatch) return FLUXBIN_ERR_UNSUPPORTED;
+    const size_t need = workspace_bytes_for(desc->M, B);
+    if (need > (size_t)FLUXBIN_STATIC_SCRATCH_BYTES) return FLUXBIN_ERR_SCRATCH_LIMIT;
+    if (need == 0)  // nothing to launch (M == 0 or B == 0): validate and return
+        return fluxbin_linear(desc, d_words, d_r, d_c, d_swords, d_rs, d_cs, d_idx, d_x, B, d_y, flags, nullptr, 0,
+                              stream);
+    void* scratch = nullptr;
+    const int sa = static_scratch_address(&scratch);
+    if (sa != FLUXBIN_OK) return sa;
+    // the previous call on this device may have left anything there
+    if (cudaMemsetAsync(scratch, 0, need, static_cast<cudaStream_t>(stream)) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return FLUXBIN_ERR_CUDA;
+    }
+    return fluxbin_linear(desc, d_words, d_r, d_c, d_swords, d_rs, d_cs, d_idx, d_x, B, d_y, flags, scratch,
+                          (size_t)FLUXBIN_STATIC_SCRATCH_BYTES, stream);
+}

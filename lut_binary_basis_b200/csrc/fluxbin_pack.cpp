@@ -60,6 +60,7 @@ const char* fluxbin_status_string(int status) {
         case FLUXBIN_ERR_SMEM_BUDGET: return "shared-memory budget exceeded";
         case FLUXBIN_ERR_WORKSPACE: return "workspace missing or too small";
         case FLUXBIN_ERR_CUDA: return "CUDA error";
+        case FLUXBIN_ERR_SCRATCH_LIMIT: return "layer too large for the static scratch";
         default: return "unknown status";
     }
 }

@@ -23,7 +23,9 @@ FLAG_EARLY_WEIGHTS = 4
 
 STATUS = {0: "FLUXBIN_OK", -1: "FLUXBIN_ERR_INVALID_ARG", -2: "FLUXBIN_ERR_BAD_SHAPE",
           -3: "FLUXBIN_ERR_MISALIGNED", -4: "FLUXBIN_ERR_UNSUPPORTED", -5: "FLUXBIN_ERR_SMEM_BUDGET",
-          -6: "FLUXBIN_ERR_WORKSPACE", -7: "FLUXBIN_ERR_CUDA"}
+          -6: "FLUXBIN_ERR_WORKSPACE", -7: "FLUXBIN_ERR_CUDA", -8: "FLUXBIN_ERR_SCRATCH_LIMIT"}
+
+STATIC_SCRATCH_BYTES = 4 << 20
 
 
 class FluxbinLibraryMissing(ImportError):
@@ -68,8 +70,9 @@ def lib():
             L.fluxbin_workspace_bytes.argtypes = [i32, i32, ctypes.POINTER(sz)]
             L.fluxbin_lut_gemv.argtypes = [i32, i32, i32, i32, i32, i32, P, P, P, P, P, i32, P, u32, P, sz, P]
             L.fluxbin_linear.argtypes = [P, P, P, P, P, P, P, P, P, i32, P, u32, P, sz, P]
+            L.fluxbin_linear_static_scratch.argtypes = [P, P, P, P, P, P, P, P, P, i32, P, u32, P]
             for f in ("fluxbin_packed_sizes", "fluxbin_pack", "fluxbin_workspace_bytes", "fluxbin_lut_gemv",
-                      "fluxbin_linear"):
+                      "fluxbin_linear", "fluxbin_linear_static_scratch"):
                 getattr(L, f).restype = ctypes.c_int
             _lib = L
     return _lib
@@ -153,6 +156,17 @@ def fluxbin_linear(desc: LayerDesc, words, r, c, swords, rs, cs, idx, x, B: int,
     _check(lib().fluxbin_linear(ctypes.byref(desc), _dptr(words), _dptr(r), _dptr(c), _dptr(swords), _dptr(rs),
                                 _dptr(cs), _dptr(idx), _dptr(x), B, _dptr(y), flags, _dptr(workspace), wsb,
                                 _stream(stream)), "fluxbin_linear")
+
+
+def fluxbin_linear_static_scratch(desc: LayerDesc, words, r, c, swords, rs, cs, idx, x, B: int, y,
+                                  flags: int = FLAG_Y_FP32, stream=None) -> None:
+    """fluxbin_linear without a workspace argument, for callers that cannot
+    allocate device memory: the split-K scratch is the library's own fixed
+    device array (STATIC_SCRATCH_BYTES per device).  Calls that may overlap on
+    the GPU share that array and must be ordered on one stream."""
+    _check(lib().fluxbin_linear_static_scratch(ctypes.byref(desc), _dptr(words), _dptr(r), _dptr(c), _dptr(swords),
+                                               _dptr(rs), _dptr(cs), _dptr(idx), _dptr(x), B, _dptr(y), flags,
+                                               _stream(stream)), "fluxbin_linear_static_scratch")
 
 
 @dataclasses.dataclass
