@@ -475,6 +475,28 @@ def time_layer(spec, B, device, l2, wid, steps=50):
             "copies": R}
 
 
+def find_layer(name):
+    from lut_binary_basis_b200 import synth
+    for wid, (_, specs, _) in synth.WORKLOADS.items():
+        for sp in specs:
+            if sp.name == name:
+                return wid, sp
+    raise SystemExit(f"unknown layer {name!r}")
+
+
+def run_one_layer(args):
+    """One layer of the workloads at one batch size (also the profiling driver)."""
+    import torch
+    import __graft_entry__
+    __graft_entry__.build()
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    wid, sp = find_layer(args.layer)
+    props = torch.cuda.get_device_properties(device)
+    l2 = getattr(props, "L2_cache_size", 126 * 2 ** 20) or 126 * 2 ** 20
+    return time_layer(sp, args.batch, device, l2, wid, steps=args.steps)
+
+
 def run_sweep(device, l2, args):
     from lut_binary_basis_b200 import synth
     out = []
@@ -522,9 +544,15 @@ def main(argv=None):
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-cublas", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
+    ap.add_argument("--layer", default=None,
+                    help="time one named layer of the workloads instead (e.g. llama7b_gate_up_11008x4096)")
+    ap.add_argument("--batch", type=int, default=1)
     args = ap.parse_args(argv)
     args.warmup = max(3, args.warmup)
     rank, local_rank, world = dist_env()
+    if args.layer:
+        print(json.dumps(run_one_layer(args)), flush=True)
+        return
     if args.impl == "reference":
         res = run_reference(args, rank, world)
     else:

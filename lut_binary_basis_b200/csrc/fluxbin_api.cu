@@ -23,40 +23,89 @@ int batch_tile(int mu, int B) {
     return B <= 1 ? 1 : (B <= 2 ? 2 : 4);
 }
 
-size_t table_smem_bytes(int mu, int bt) { return (size_t)bt * ((size_t)1 << mu) * 256u; }
+// Tables plus the double-buffered activation products (see fluxbin_kernel.cuh).
+size_t table_smem_bytes(int mu, int bt) {
+    return (size_t)bt * ((size_t)1 << mu) * 256u + 2u * (size_t)bt * 32u * (size_t)mu * sizeof(float);
+}
+// Cluster reduction buffer: one fp32 partial per row of the CTA and batch row.
+size_t red_smem_bytes(int bt) { return (size_t)bt * kRowsPerCta * sizeof(float); }
 
-struct LaunchInfo {
-    int blocks_per_sm = 0;
+struct DeviceInfo {
     int sm_count = 0;
     int max_smem = 0;
 };
 
-std::mutex g_mu;
-std::unordered_map<uint64_t, LaunchInfo> g_info;
+struct FuncInfo {
+    int blocks_per_sm = 0;  // with the reduction buffer
+};
 
-int launch_info(KernelFn fn, size_t smem, LaunchInfo* out) {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return FLUXBIN_ERR_CUDA;
-    const uint64_t key = (reinterpret_cast<uint64_t>(fn) << 8) ^ (uint64_t)dev;
-    std::lock_guard<std::mutex> lock(g_mu);
-    auto it = g_info.find(key);
-    if (it != g_info.end()) {
+std::mutex g_mu;
+std::unordered_map<int, DeviceInfo> g_dev;
+std::unordered_map<uint64_t, FuncInfo> g_func;
+std::unordered_map<uint64_t, int> g_clusters;
+
+int device_info(int dev, DeviceInfo* out) {
+    auto it = g_dev.find(dev);
+    if (it != g_dev.end()) {
         *out = it->second;
         return FLUXBIN_OK;
     }
-    LaunchInfo li;
-    if (cudaDeviceGetAttribute(&li.sm_count, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&li.max_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
+    DeviceInfo di;
+    if (cudaDeviceGetAttribute(&di.sm_count, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&di.max_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
         return FLUXBIN_ERR_CUDA;
-    if ((size_t)li.max_smem < smem + 1024) return FLUXBIN_ERR_SMEM_BUDGET;
-    if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
-        return FLUXBIN_ERR_CUDA;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&li.blocks_per_sm, fn, kThreads, smem) != cudaSuccess)
-        return FLUXBIN_ERR_CUDA;
-    if (li.blocks_per_sm < 1) return FLUXBIN_ERR_SMEM_BUDGET;
-    g_info.emplace(key, li);
-    *out = li;
+    g_dev.emplace(dev, di);
+    *out = di;
     return FLUXBIN_OK;
+}
+
+// Per-function, per-device set-up: opt in to the dynamic shared memory of the
+// largest launch and to non-portable cluster sizes; occupancy.
+int func_info(KernelFn fn, int dev, int mu, int bt, const DeviceInfo& di, FuncInfo* out) {
+    const uint64_t key = (reinterpret_cast<uint64_t>(fn) << 8) ^ (uint64_t)dev;
+    auto it = g_func.find(key);
+    if (it != g_func.end()) {
+        *out = it->second;
+        return FLUXBIN_OK;
+    }
+    FuncInfo fi;
+    const size_t smem_max = table_smem_bytes(mu, bt) + red_smem_bytes(bt);
+    if ((size_t)di.max_smem < smem_max) return FLUXBIN_ERR_SMEM_BUDGET;
+    if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_max) != cudaSuccess ||
+        cudaFuncSetAttribute(fn, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&fi.blocks_per_sm, fn, kThreads, smem_max) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return FLUXBIN_ERR_CUDA;
+    }
+    if (fi.blocks_per_sm < 1) return FLUXBIN_ERR_SMEM_BUDGET;
+    g_func.emplace(key, fi);
+    *out = fi;
+    return FLUXBIN_OK;
+}
+
+// How many clusters of `csize` CTAs can be resident at once (0: none).
+int max_active_clusters(KernelFn fn, int dev, int csize, size_t smem) {
+    const uint64_t key = (reinterpret_cast<uint64_t>(fn) << 12) ^ ((uint64_t)dev << 8) ^ (uint64_t)csize;
+    auto it = g_clusters.find(key);
+    if (it != g_clusters.end()) return it->second;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)csize);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)csize;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, fn, &cfg) != cudaSuccess) {
+        (void)cudaGetLastError();
+        n = 0;
+    }
+    g_clusters.emplace(key, n);
+    return n;
 }
 
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
@@ -68,6 +117,56 @@ struct BranchIn {
     const int32_t* gather;
     int32_t ncols, nb, rgroup;
 };
+
+// Launch shape: the split of the units over CTAs and how it is reduced.
+struct Plan {
+    int n_rg = 1;
+    int n_ks = 1;
+    bool cluster = false;
+};
+
+// Row groups of 512 rows times batch chunks fix the number of CTA groups; the
+// units are split over up to 16 CTAs per group forming a cluster whose
+// partials are reduced in DSMEM.  A layer whose packed words come to at most
+// kSmallLayerBytesPerSm per SM gets at most one CTA per SM, so that the CTAs
+// of the next call on the stream fit beside them and fetch their own words
+// while this call finishes (programmatic dependent launch); larger layers
+// fill every CTA slot.  Every cluster must be resident at once.  When that
+// leaves most SMs idle (few rows, long rows) the units are split as widely
+// as the SMs allow and reduced through the workspace.
+constexpr int64_t kSmallLayerBytesPerSm = 96 * 1024;
+
+Plan make_plan(KernelFn fn, int dev, int mu, int bt, int64_t Ms, int64_t U, int n_bc, const DeviceInfo& di,
+               const FuncInfo& fi) {
+    Plan p;
+    p.n_rg = (int)((Ms + kSlabsPerCta - 1) / kSlabsPerCta);
+    const int64_t groups = (int64_t)p.n_rg * n_bc;
+    const int64_t layer_bytes = Ms * U * 128 * mu;
+    const bool small = layer_bytes <= kSmallLayerBytesPerSm * di.sm_count;
+    const int64_t slots = (int64_t)di.sm_count * (small ? 1 : fi.blocks_per_sm);
+    int64_t want = slots / groups;
+    if (want > U) want = U;
+    if (want > kMaxCluster) want = kMaxCluster;
+    const size_t smem = table_smem_bytes(mu, bt) + red_smem_bytes(bt);
+    for (int64_t ks = want; ks >= 2; --ks) {
+        if (groups * ks * 2 < di.sm_count) break;  // too few CTAs: use the workspace instead
+        if (max_active_clusters(fn, dev, (int)ks, smem) >= groups) {
+            p.n_ks = (int)ks;
+            p.cluster = true;
+            return p;
+        }
+    }
+    if (groups * 2 >= di.sm_count || U <= 1) {
+        p.n_ks = 1;  // enough row groups: no split at all
+        return p;
+    }
+    int64_t ks = (slots + groups / 2) / groups;
+    if (ks > U) ks = U;
+    if (ks < 1) ks = 1;
+    p.n_ks = (int)ks;
+    p.cluster = false;
+    return p;
+}
 
 int run(int32_t M, int32_t N, int mu, const BranchIn& g, const BranchIn* s, const uint16_t* d_x, int32_t B,
         void* d_y, uint32_t flags, void* ws, size_t ws_bytes, void* stream) {
@@ -89,11 +188,12 @@ int run(int32_t M, int32_t N, int mu, const BranchIn& g, const BranchIn* s, cons
     const int bt = batch_tile(mu, B);
     KernelFn fn = mu == 8 ? select_kernel_mu8(g.nb, nb1, bt) : select_kernel_mu4(g.nb, nb1, bt);
     if (!fn) return FLUXBIN_ERR_UNSUPPORTED;
-    const size_t smem = table_smem_bytes(mu, bt);
-    LaunchInfo li;
-    int st = launch_info(fn, smem, &li);
-    if (st != FLUXBIN_OK) return st;
 
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return FLUXBIN_ERR_CUDA;
+    DeviceInfo di;
+    FuncInfo fi;
+    Plan plan;
     KernelArgs a = {};
     const BranchIn* in[2] = {&g, nb1 ? s : nullptr};
     for (int q = 0; q < 2; ++q) {
@@ -108,24 +208,29 @@ int run(int32_t M, int32_t N, int mu, const BranchIn& g, const BranchIn* s, cons
         o.rgroup = in[q]->rgroup;
         o.ngroups = in[q]->rgroup > 0 ? (in[q]->ncols + in[q]->rgroup - 1) / in[q]->rgroup : 0;
     }
+    a.Ms = (int32_t)row_slabs(M);
+    const int n_bc = (B + bt - 1) / bt;
+    const int64_t U = (int64_t)a.br[0].units + a.br[1].units;
+    {
+        std::lock_guard<std::mutex> lock(g_mu);
+        int st = device_info(dev, &di);
+        if (st != FLUXBIN_OK) return st;
+        st = func_info(fn, dev, mu, bt, di, &fi);
+        if (st != FLUXBIN_OK) return st;
+        plan = make_plan(fn, dev, mu, bt, a.Ms, U, n_bc, di, fi);
+    }
     a.x = reinterpret_cast<const __half*>(d_x);
     a.y = d_y;
     a.M = M;
     a.N = N;
     a.B = B;
-    a.Ms = (int32_t)row_slabs(M);
     a.Mp = a.Ms * kLanes;
-    a.n_rg = (a.Ms + kSlabsPerCta - 1) / kSlabsPerCta;
-    a.n_bc = (B + bt - 1) / bt;
+    a.n_rg = plan.n_rg;
+    a.n_bc = n_bc;
+    a.n_ks = plan.n_ks;
+    a.cluster = plan.cluster ? 1 : 0;
     a.flags = flags;
-    const int64_t U = (int64_t)a.br[0].units + a.br[1].units;
-    const int64_t groups = (int64_t)a.n_rg * a.n_bc;
-    const int64_t target = (int64_t)li.sm_count * li.blocks_per_sm;
-    int64_t ks = (target + groups / 2) / groups;
-    if (ks > U) ks = U;
-    if (ks < 1) ks = 1;
-    a.n_ks = (int32_t)ks;
-    if (a.n_ks > 1) {
+    if (a.n_ks > 1 && !plan.cluster) {
         const size_t need = workspace_bytes_for(M, B);
         if (!ws || ws_bytes < need) return FLUXBIN_ERR_WORKSPACE;
         if (!aligned(ws, 16)) return FLUXBIN_ERR_MISALIGNED;
@@ -135,15 +240,22 @@ int run(int32_t M, int32_t N, int mu, const BranchIn& g, const BranchIn* s, cons
     }
 
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)(groups * a.n_ks));
+    cfg.gridDim = dim3((unsigned)((int64_t)a.n_rg * a.n_bc * a.n_ks));
     cfg.blockDim = dim3(kThreads);
-    cfg.dynamicSmemBytes = smem;
+    cfg.dynamicSmemBytes = table_smem_bytes(mu, bt) + (plan.cluster ? red_smem_bytes(bt) : 0);
     cfg.stream = static_cast<cudaStream_t>(stream);
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
+    if (plan.cluster) {
+        attr[1].id = cudaLaunchAttributeClusterDimension;
+        attr[1].val.clusterDim.x = (unsigned)a.n_ks;
+        attr[1].val.clusterDim.y = 1;
+        attr[1].val.clusterDim.z = 1;
+        cfg.numAttrs = 2;
+    }
     if (cudaLaunchKernelEx(&cfg, fn, a) != cudaSuccess) {
         (void)cudaGetLastError();
         return FLUXBIN_ERR_CUDA;

@@ -6,15 +6,15 @@ namespace fluxbin {
 using KernelFn = void (*)(KernelArgs);
 
 namespace {
-template <int BT, int MINB>
+template <int BT>
 KernelFn pick(int nb0, int nb1) {
-#define FB_NB1(NB0)                                                   \
-    switch (nb1) {                                                    \
-        case 0: return &fluxbin_lut_kernel<8, NB0, 0, BT, MINB>;  \
-        case 1: return &fluxbin_lut_kernel<8, NB0, 1, BT, MINB>;  \
-        case 2: return &fluxbin_lut_kernel<8, NB0, 2, BT, MINB>;  \
-        case 4: return &fluxbin_lut_kernel<8, NB0, 4, BT, MINB>;  \
-        default: return nullptr;                                      \
+#define FB_NB1(NB0)                                             \
+    switch (nb1) {                                              \
+        case 0: return &fluxbin_lut_kernel<8, NB0, 0, BT>;  \
+        case 1: return &fluxbin_lut_kernel<8, NB0, 1, BT>;  \
+        case 2: return &fluxbin_lut_kernel<8, NB0, 2, BT>;  \
+        case 4: return &fluxbin_lut_kernel<8, NB0, 4, BT>;  \
+        default: return nullptr;                                \
     }
     switch (nb0) {
         case 1: FB_NB1(1)
@@ -26,11 +26,10 @@ KernelFn pick(int nb0, int nb1) {
 }
 }  // namespace
 
-// Tables of one batch row take 64 KiB (two 32 KiB halves): two CTAs per SM
-// for one batch row per CTA, one CTA per SM for two.
+// Tables of one batch row take 64 KiB (two 32 KiB halves).
 KernelFn select_kernel_mu8(int nb0, int nb1, int bt) {
-    if (bt == 1) return pick<1, 2>(nb0, nb1);
-    if (bt == 2) return pick<2, 1>(nb0, nb1);
+    if (bt == 1) return pick<1>(nb0, nb1);
+    if (bt == 2) return pick<2>(nb0, nb1);
     return nullptr;
 }
 

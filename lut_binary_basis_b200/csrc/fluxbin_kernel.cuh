@@ -7,36 +7,48 @@
 //
 // Work decomposition.  The packed signs of a branch are cut into units of
 // P = 32/nb sub-vectors per base (32 tables per unit) and into row slabs of 32
-// rows (include/fluxbin.h, "Packed sign layout").  A CTA of 8 warps owns 1024
-// rows (each warp 4 slabs, each lane one row per slab), one batch chunk of BT
-// rows and a contiguous range of units (a split of the reduction dimension).
-// For every unit it
-//   1. builds the unit's 32 tables per batch row in shared memory: the column
-//      scale is fused into the activation (v = c (.) x, the salient branch
-//      gathering x through its column map) and the 2^mu signed partial sums of
-//      each sub-vector are enumerated in Gray-code order, one fp32 add per entry
-//      (LUT building with scale fusion, Section 3; Appendix C.1);
-//   2. has every lane stream its rows' packed words with 128-bit loads
-//      (prefetched one unit ahead into registers) and, at each of 32 steps,
-//      turn the next mu-bit pattern into a shared-memory address and add the
-//      table entry into an fp32 register accumulator.  The layout's visit
-//      order puts the 32 lanes of a warp on 32 different tables, each in its
-//      own bank, so the random-looking lookups never conflict;
-//   3. after its last unit, multiplies each accumulator by its row scale (per
-//      row, or per row and column block after every unit), and either stores
-//      y or adds its partial into an fp32 workspace, the last CTA of a row group
-//      to arrive writing y and re-zeroing the workspace (split-K reduction; the
-//      pages use global atomics across K tiles, Appendix E.3).
+// rows (include/fluxbin.h, "Packed sign layout").  A CTA of 8 warps owns 512
+// rows (each warp two slabs, each lane one row per slab), one batch chunk of
+// BT rows and a contiguous range of units (a split of the reduction
+// dimension).  For every unit it
+//   1. forms the unit's 32*mu activation products v = c (.) x once, one slot
+//      per thread, two units ahead of their use (column scale fused into the
+//      activation; the salient branch gathers x through its column map),
+//      parked in a small double-buffered shared array;
+//   2. builds the unit's 32 tables per batch row from them: the 2^mu signed
+//      partial sums of every sub-vector, enumerated in Gray-code order, one
+//      fp32 add per entry (LUT building with scale fusion, Section 3;
+//      Appendix C.1);
+//   3. has every lane stream its rows' packed words with 128-bit loads,
+//      requested two units ahead into registers, and at each of 32 steps turn
+//      the next mu-bit pattern into a shared-memory address (one byte-permute
+//      with a per-lane offset word) and add the table entry into an fp32
+//      register.  The layout's visit order puts the 32 lanes of a warp on 32
+//      different tables, each in its own bank: the lookups never conflict;
+//   4. after its last unit multiplies each accumulator by its row scale (per
+//      row, or per row and column block after every unit) and reduces the
+//      split-K partials: inside a thread-block cluster through distributed
+//      shared memory (fixed order, no global traffic), or, when the reduction
+//      is wider than a cluster, through an fp32 workspace where the last CTA to
+//      arrive writes y (the pages reduce across K tiles with global atomics,
+//      Appendix E.3).
+// Everything that belongs to the layer (packed words, scales, column map) is
+// requested before the kernel waits for its predecessor on the stream
+// (programmatic dependent launch); only activations, outputs and workspace
+// are touched after that wait.
 //
-// Tables live in rows of 256 bytes: entry e of the tables for batch row b and
-// unit parity h sits at b*2^mu*256 + e*256 + h*128 + bank*4, so consecutive
-// units alternate between the two 128-byte halves (double buffering with one
-// barrier per unit) and, for mu = 8, a byte-permute of the packed word with a
-// per-lane offset register yields the whole address in one instruction.
+// Shared memory (byte offsets from the start of the dynamic allocation):
+//   tables  BT * 2^mu * 256: entry e of the tables of batch row b for unit
+//           parity h at b*2^mu*256 + e*256 + h*128 + bank*4 (consecutive units
+//           alternate halves: double buffering with one barrier per unit)
+//   vbuf    2 * BT * 32*mu floats: [parity][b][bank][t] activation products
+//   red     BT * 512 floats: partial sums for the cluster reduction
 #pragma once
 
 #include <cuda_fp16.h>
 #include <stdint.h>
+
+#include <type_traits>
 
 #include "fluxbin_layout.h"
 
@@ -61,6 +73,7 @@ struct KernelArgs {
     int32_t Ms;             // row slabs
     int32_t Mp;             // Ms * 32
     int32_t n_rg, n_ks, n_bc;
+    int32_t cluster;        // 1: the n_ks CTAs of a row group form a cluster and reduce in DSMEM
     uint32_t flags;
     float* ws_acc;          // [B][Mp] split-K partial sums (zero between calls)
     unsigned int* ws_cnt;   // [n_rg * n_bc] arrival counters (zero between calls)
@@ -70,14 +83,48 @@ constexpr uint32_t kFlagAccumulate = 1u;
 constexpr uint32_t kFlagYFp32 = 2u;
 constexpr uint32_t kFlagEarlyWeights = 4u;
 
-template <int MU>
+template <int MU, int BT>
 struct Geom {
     static constexpr int kEntries = 1 << MU;
-    static constexpr int kPairBytes = kEntries * 256;  // both halves of one batch row
-    static constexpr int kVecs = MU / 4;                // uint4 per lane per unit
+    static constexpr int kPairBytes = kEntries * 256;      // both halves of one batch row
+    static constexpr int kVecs = MU / 4;                    // uint4 per lane per unit
+    static constexpr int kLo = MU == 8 ? 4 : 2;             // entry bits enumerated per build block
+    static constexpr int kBlocks = 1 << (MU - kLo);         // build blocks per batch row
+    static constexpr int kSlots = 32 * MU;                  // activation products per unit and batch row
+    static constexpr int kTableBytes = BT * kPairBytes;
+    static constexpr int kVbufOff = kTableBytes;
+    static constexpr int kVbufBytes = 2 * BT * kSlots * 4;
+    static constexpr int kRedOff = kVbufOff + kVbufBytes;
+    static constexpr int kRedBytes = BT * kRowsPerCta * 4;
 };
 
+// Byte offsets (bank * 4) of the tables lane L visits at steps 3r, 3r+1, 3r+2,
+// packed into bytes 0..2 of word [nb index][r][L]; byte 3 is zero.
+struct OffsetTable {
+    uint32_t w[3][11][32];
+};
+constexpr OffsetTable make_offset_table() {
+    OffsetTable t{};
+    for (int nbi = 0; nbi < 3; ++nbi)
+        for (int r = 0; r < 11; ++r)
+            for (int L = 0; L < 32; ++L) {
+                uint32_t v = 0;
+                for (int m = 0; m < 3; ++m) {
+                    const int q = 3 * r + m;
+                    if (q < 32) v |= (uint32_t)(visit_bank(L, q, 1 << nbi) * 4) << (8 * m);
+                }
+                t.w[nbi][r][L] = v;
+            }
+    return t;
+}
+__device__ const OffsetTable kOffsetTable = make_offset_table();
+
+template <int NB>
+constexpr int nb_index() { return NB == 1 ? 0 : (NB == 2 ? 1 : 2); }
+
 extern __shared__ __align__(1024) unsigned char fb_smem[];
+
+__device__ __forceinline__ uint32_t smem_base() { return (uint32_t)__cvta_generic_to_shared(fb_smem); }
 
 __device__ __forceinline__ uint4 ld_stream(const uint4* p) {
     uint4 v;
@@ -86,66 +133,100 @@ __device__ __forceinline__ uint4 ld_stream(const uint4* p) {
     return v;
 }
 
-__device__ __forceinline__ float lds_f32(uint32_t byte_off) {
-    return *reinterpret_cast<const float*>(fb_smem + byte_off);
+// Shared-memory access by 32-bit shared address (+ a constant byte offset).
+template <int OFF>
+__device__ __forceinline__ float lds_f32(uint32_t addr) {
+    float v;
+    asm volatile("ld.shared.f32 %0, [%1+%2];" : "=f"(v) : "r"(addr), "n"(OFF));
+    return v;
+}
+__device__ __forceinline__ float4 lds_f32x4(uint32_t addr) {
+    float4 v;
+    asm volatile("ld.shared.v4.f32 {%0,%1,%2,%3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(addr));
+    return v;
+}
+__device__ __forceinline__ void sts_f32(uint32_t addr, float v) {
+    asm volatile("st.shared.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
+}
+template <int OFF>
+__device__ __forceinline__ void sts_f32_at(uint32_t addr, float v) {
+    asm volatile("st.shared.f32 [%0+%1], %2;" ::"r"(addr), "n"(OFF), "f"(v) : "memory");
 }
 
-__device__ __forceinline__ void sts_f32(uint32_t byte_off, float v) {
-    *reinterpret_cast<float*>(fb_smem + byte_off) = v;
+// Two fp32 values in one 64-bit register, added pairwise by one instruction.
+__device__ __forceinline__ uint64_t pack_f32x2(float lo, float hi) {
+    uint64_t x;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(x) : "f"(lo), "f"(hi));
+    return x;
+}
+__device__ __forceinline__ uint64_t add_f32x2(uint64_t x, uint64_t y) {
+    uint64_t z;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(z) : "l"(x), "l"(y));
+    return z;
+}
+__device__ __forceinline__ float sum_f32x2(uint64_t x) {
+    float lo, hi;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(x));
+    return lo + hi;
+}
+
+// Ask the L2 to fetch [p, p + bytes) from HBM (bytes a multiple of 16).
+__device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
 }
 
 __device__ __forceinline__ void red_add_f32(float* p, float v) {
     asm volatile("red.global.add.f32 [%0], %1;" ::"l"(p), "f"(v) : "memory");
 }
 
-// Per-lane byte offsets of the 32 tables visited at steps q = 0..31, packed
-// three per register with a zero top byte (for mu = 8 address generation).
-template <int NB>
-__device__ __forceinline__ void make_offsets_packed(int lane, uint32_t (&offp)[11]) {
-#pragma unroll
-    for (int r = 0; r < 11; ++r) {
-        uint32_t v = 0;
-#pragma unroll
-        for (int m = 0; m < 3; ++m) {
-            const int q = 3 * r + m;
-            if (q < 32) v |= (uint32_t)(visit_bank(lane, q, NB) * 4) << (8 * m);
-        }
-        offp[r] = v;
-    }
+__device__ __forceinline__ void cluster_sync_all() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
-template <int NB>
-__device__ __forceinline__ void make_offsets_full(int lane, uint32_t (&offr)[32]) {
-#pragma unroll
-    for (int q = 0; q < 32; ++q) offr[q] = (uint32_t)(visit_bank(lane, q, NB) * 4);
+__device__ __forceinline__ uint32_t cluster_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+// Load a float from the same shared-memory offset in CTA `rank` of the cluster.
+__device__ __forceinline__ float ld_dsmem_f32(uint32_t local_smem_addr, uint32_t rank) {
+    uint32_t ra;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(local_smem_addr), "r"(rank));
+    float v;
+    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(ra) : "memory");
+    return v;
 }
 
 template <int MU>
-struct Offsets;
-template <>
-struct Offsets<8> {
+struct Offsets {
     uint32_t o[11];
     template <int NB>
-    __device__ __forceinline__ void make(int lane) { make_offsets_packed<NB>(lane, o); }
-    // (pattern byte q%4 of w) << 8 | offset of step q
-    __device__ __forceinline__ uint32_t addr(uint32_t w, int q) const {
-        return __byte_perm(w, o[q / 3], (uint32_t)(4 + q % 3) | ((uint32_t)(q % 4) << 4) | 0x7700u);
+    __device__ __forceinline__ void load(int lane) {
+#pragma unroll
+        for (int r = 0; r < 11; ++r) o[r] = __ldg(&kOffsetTable.w[nb_index<NB>()][r][lane]);
     }
-};
-template <>
-struct Offsets<4> {
-    uint32_t o[32];
-    template <int NB>
-    __device__ __forceinline__ void make(int lane) { make_offsets_full<NB>(lane, o); }
-    // (nibble q%8 of w) << 8 | offset of step q
+    // table byte offset of the entry step q selects: (pattern << 8) | bank*4
     __device__ __forceinline__ uint32_t addr(uint32_t w, int q) const {
-        const int n = q % 8;
-        const uint32_t e8 = (n >= 2) ? ((w >> (4 * n - 8)) & 0xF00u) : ((w << (8 - 4 * n)) & 0xF00u);
-        return e8 | o[q];
+        if constexpr (MU == 8) {
+            return __byte_perm(w, o[q / 3], (uint32_t)(4 + q % 3) | ((uint32_t)(q % 4) << 4) | 0x7700u);
+        } else {
+            const int n = q % 8;
+            const uint32_t e8 = (n >= 2) ? ((w >> (4 * n - 8)) & 0xF00u) : ((w << (8 - 4 * n)) & 0xF00u);
+            return __byte_perm(e8, o[q / 3], (uint32_t)(4 + q % 3) | 0x7710u);
+        }
     }
 };
 
-// Index of the lowest set bit of i > 0 (the bit that flips between Gray codes i-1 and i).
+// Calls f(std::integral_constant<int, I>) for I = 0 .. N-1 (compile-time indices).
+template <int I, int N, typename F>
+__device__ __forceinline__ void static_for(F&& f) {
+    if constexpr (I < N) {
+        f(std::integral_constant<int, I>{});
+        static_for<I + 1, N>(f);
+    }
+}
+
 __host__ __device__ __forceinline__ constexpr int lowest_bit(int i) {
     int t = 0;
     while (!((i >> t) & 1)) ++t;
@@ -156,74 +237,122 @@ __device__ __forceinline__ uint32_t word_of(const uint4& v, int i) {
     return i == 0 ? v.x : (i == 1 ? v.y : (i == 2 ? v.z : v.w));
 }
 
-// 32 lookup-accumulate steps of one lane for one row slab and unit.
+// 32 lookup-accumulate steps of one lane for one row slab and unit.  Steps
+// q and q+1 always feed the same accumulator; their entries are added as a
+// pair (one paired fp32 add per two lookups) and folded into acc at the end.
 template <int MU, int NB, int HALF, int BT>
-__device__ __forceinline__ void lookup_unit(const uint4 (&w)[Geom<MU>::kVecs], const Offsets<MU>& off,
-                                            float (&acc)[BT][NB]) {
+__device__ __forceinline__ void lookup_unit(const uint4 (&w)[Geom<MU, BT>::kVecs], const Offsets<MU>& off,
+                                            uint32_t tbase, float (&acc)[BT][NB]) {
     constexpr int P = 32 / NB;
     constexpr int kStepsPerWord = 32 / MU;
+    uint64_t pair[BT][NB];
 #pragma unroll
-    for (int q = 0; q < 32; ++q) {
-        const int wi = q / kStepsPerWord;
-        const uint32_t word = word_of(w[wi / 4], wi % 4);
-        const uint32_t a = off.addr(word, q);
+    for (int b = 0; b < BT; ++b)
 #pragma unroll
-        for (int b = 0; b < BT; ++b)
-            acc[b][q / P] += lds_f32(a + (uint32_t)(b * Geom<MU>::kPairBytes + HALF * 128));
+        for (int i = 0; i < NB; ++i) pair[b][i] = 0ull;
+#pragma unroll
+    for (int q = 0; q < 32; q += 2) {
+        const int wi0 = q / kStepsPerWord, wi1 = (q + 1) / kStepsPerWord;
+        const uint32_t a0 = tbase + off.addr(word_of(w[wi0 / 4], wi0 % 4), q);
+        const uint32_t a1 = tbase + off.addr(word_of(w[wi1 / 4], wi1 % 4), q + 1);
+        static_for<0, BT>([&](auto bc) {
+            constexpr int b = decltype(bc)::value;
+            constexpr int OFF = b * Geom<MU, BT>::kPairBytes + HALF * 128;
+            const float f0 = lds_f32<OFF>(a0);
+            const float f1 = lds_f32<OFF>(a1);
+            pair[b][q / P] = add_f32x2(pair[b][q / P], pack_f32x2(f0, f1));
+        });
     }
+#pragma unroll
+    for (int b = 0; b < BT; ++b)
+#pragma unroll
+        for (int i = 0; i < NB; ++i) acc[b][i] += sum_f32x2(pair[b][i]);
+}
+
+// The activation-product slot a thread owns: bank c = s / mu, bit t = s % mu.
+struct SlotStatic {
+    float c;   // column scale (0 for padding and out-of-range columns)
+    int col;   // activation column (-1 for padding)
+};
+
+template <int MU, int NB0, int NB1>
+__device__ __forceinline__ SlotStatic slot_static(const KernelArgs& a, int u, int s) {
+    SlotStatic r{0.f, -1};
+    const bool br1 = NB1 > 0 && u >= a.br[0].units;
+    // select fields one by one (a reference chosen at run time would force a
+    // local copy of the kernel parameters)
+    const __half* cptr = br1 ? a.br[1].c : a.br[0].c;
+    const int32_t* gptr = br1 ? a.br[1].gather : a.br[0].gather;
+    const int ncols = br1 ? a.br[1].ncols : a.br[0].ncols;
+    const int nb = br1 ? (NB1 > 0 ? NB1 : 1) : NB0;
+    const int P = 32 / nb;
+    const int ul = br1 ? u - a.br[0].units : u;
+    const int cb = s / MU, t = s % MU;
+    const int k = cb / P, j = cb % P;
+    const int64_t n = ((int64_t)ul * P + j) * MU + t;
+    if (n < ncols) {
+        const int cc = gptr ? __ldg(gptr + n) : (int)n;
+        if (cc >= 0 && cc < a.N) {
+            r.c = __half2float(cptr[(int64_t)k * ncols + n]);
+            r.col = cc;
+        }
+    }
+    return r;
+}
+
+template <int BT>
+__device__ __forceinline__ void slot_x(const KernelArgs& a, int b0, int col, __half (&xv)[BT]) {
+#pragma unroll
+    for (int b = 0; b < BT; ++b)
+        xv[b] = (col >= 0 && b0 + b < a.B) ? a.x[(int64_t)(b0 + b) * a.N + col] : __float2half(0.f);
+}
+
+template <int MU, int BT>
+__device__ __forceinline__ void store_products(uint32_t sbase, int parity, int s, float c, const __half (&xv)[BT]) {
+#pragma unroll
+    for (int b = 0; b < BT; ++b)
+        sts_f32(sbase + Geom<MU, BT>::kVbufOff + ((parity * BT + b) * Geom<MU, BT>::kSlots + s) * 4,
+                c * __half2float(xv[b]));
 }
 
 // Tables of one unit for BT batch rows.  Lane = bank = (base k, sub-vector j).
-template <int MU, int NB, int HALF, int BT>
-__device__ __forceinline__ void build_unit(const KernelArgs& a, const BranchArgs& br, int ul, int b0,
-                                           int warp, int lane) {
-    constexpr int P = 32 / NB;
-    constexpr int LO = MU < 5 ? MU : 5;        // bits enumerated in Gray-code order
-    constexpr int NBLK = 1 << (MU - LO);       // entry blocks per batch row
-    const int k = lane / P, j = lane % P;
-    const int64_t n0 = ((int64_t)ul * P + j) * MU;
-    float cv[MU];
-    int col[MU];
-#pragma unroll
-    for (int t = 0; t < MU; ++t) {
-        const int64_t n = n0 + t;
-        cv[t] = 0.f;
-        col[t] = 0;
-        if (n < br.ncols) {
-            const int cc = br.gather ? __ldg(br.gather + n) : (int)n;
-            if (cc >= 0 && cc < a.N) {
-                cv[t] = __half2float(br.c[(int64_t)k * br.ncols + n]);
-                col[t] = cc;
-            }
-        }
-    }
+template <int MU, int HALF, int BT>
+__device__ __forceinline__ void build_unit(uint32_t sbase, int warp, int lane) {
+    using G = Geom<MU, BT>;
+    constexpr int LO = G::kLo;
+    constexpr int NBLK = G::kBlocks;
     for (int z = warp; z < BT * NBLK; z += kWarps) {
         const int bl = z / NBLK, hi = z % NBLK;
-        const int bb = b0 + bl;
         float v[MU];
+        const uint32_t va = sbase + G::kVbufOff + ((HALF * BT + bl) * G::kSlots + lane * MU) * 4;
 #pragma unroll
-        for (int t = 0; t < MU; ++t)
-            v[t] = (bb < a.B && cv[t] != 0.f) ? cv[t] * __half2float(a.x[(int64_t)bb * a.N + col[t]]) : 0.f;
+        for (int h = 0; h < MU / 4; ++h) {
+            const float4 f = lds_f32x4(va + 16 * h);
+            v[4 * h] = f.x;
+            v[4 * h + 1] = f.y;
+            v[4 * h + 2] = f.z;
+            v[4 * h + 3] = f.w;
+        }
         float T = 0.f;
 #pragma unroll
         for (int t = LO; t < MU; ++t) T += ((hi >> (t - LO)) & 1) ? v[t] : -v[t];
 #pragma unroll
         for (int t = 0; t < LO; ++t) T -= v[t];
-        const uint32_t base = (uint32_t)(bl * Geom<MU>::kPairBytes + HALF * 128 + lane * 4);
-        sts_f32(base + (uint32_t)(hi << LO) * 256u, T);
-#pragma unroll
-        for (int i = 1; i < (1 << LO); ++i) {
-            const int t = lowest_bit(i);
-            const int g = i ^ (i >> 1);
+        const uint32_t base = sbase + (uint32_t)(bl * G::kPairBytes + lane * 4) + (uint32_t)(hi << LO) * 256u;
+        sts_f32_at<HALF * 128>(base, T);
+        static_for<1, (1 << LO)>([&](auto ic) {
+            constexpr int i = decltype(ic)::value;
+            constexpr int t = lowest_bit(i);
+            constexpr int g = i ^ (i >> 1);
             T += ((g >> t) & 1) ? 2.f * v[t] : -2.f * v[t];
-            sts_f32(base + (uint32_t)((hi << LO) | g) * 256u, T);
-        }
+            sts_f32_at<g * 256 + HALF * 128>(base, T);
+        });
     }
 }
 
-template <int MU>
+template <int MU, int BT>
 __device__ __forceinline__ void load_unit_slab(const KernelArgs& a, int u, int sl, int lane,
-                                               uint4 (&w)[Geom<MU>::kVecs]) {
+                                               uint4 (&w)[Geom<MU, BT>::kVecs]) {
     const bool br1 = u >= a.br[0].units;
     const int ul = br1 ? u - a.br[0].units : u;
     const uint4* base = br1 ? a.br[1].words : a.br[0].words;
@@ -231,35 +360,53 @@ __device__ __forceinline__ void load_unit_slab(const KernelArgs& a, int u, int s
     if (sl < a.Ms) {
         const uint4* p = base + ((int64_t)sl * U + ul) * (8 * MU) + lane;
 #pragma unroll
-        for (int h = 0; h < Geom<MU>::kVecs; ++h) w[h] = ld_stream(p + h * 32);
+        for (int h = 0; h < Geom<MU, BT>::kVecs; ++h) w[h] = ld_stream(p + h * 32);
     } else {
 #pragma unroll
-        for (int h = 0; h < Geom<MU>::kVecs; ++h) w[h] = make_uint4(0, 0, 0, 0);
+        for (int h = 0; h < Geom<MU, BT>::kVecs; ++h) w[h] = make_uint4(0, 0, 0, 0);
     }
 }
 
-// One unit of branch BR: build its tables, then every slab's lookups, with
-// the next unit's packed words requested as soon as a slab's registers free up.
-template <int MU, int BR, int NB, int HALF, int BT>
+// Per-thread state of the activation-product pipeline: the next unit's
+// products (column scale and activations loaded) and the column of the unit
+// after it (layer data loaded).
+template <int BT>
+struct ProductPipe {
+    float c1;
+    __half x1[BT];
+    float c2;
+    int col2;
+};
+
+template <int MU, int BT>
+struct WeightRegs {
+    uint4 w[2][kSlabsPerWarp][Geom<MU, BT>::kVecs];
+};
+
+// One unit of branch BR: build its tables, form the next unit's products and
+// request the inputs two units ahead, then every slab's lookups, refilling
+// each slab's registers with the unit two ahead as soon as they are consumed.
+template <int MU, int BR, int NB, int HALF, int BT, int NB0, int NB1>
 __device__ __forceinline__ void unit_step(const KernelArgs& a, int u, int u_end, int ul, int b0, int slab0,
-                                          int warp, int lane, const Offsets<MU>& off,
-                                          uint4 (&wb)[kSlabsPerWarp][Geom<MU>::kVecs],
+                                          int warp, int lane, int tid, uint32_t sbase, const Offsets<MU>& off,
+                                          ProductPipe<BT>& pp, WeightRegs<MU, BT>& wb,
                                           float (&acc)[kSlabsPerWarp][BT][NB],
                                           float (&tot)[kSlabsPerWarp][BT]) {
     const BranchArgs& br = a.br[BR];
-    build_unit<MU, NB, HALF, BT>(a, br, ul, b0, warp, lane);
-    __syncthreads();
-#pragma unroll
-    for (int rs = 0; rs < kSlabsPerWarp; ++rs) {
-        uint4 cur[Geom<MU>::kVecs];
-#pragma unroll
-        for (int h = 0; h < Geom<MU>::kVecs; ++h) cur[h] = wb[rs][h];
-        if (u + 1 < u_end) load_unit_slab<MU>(a, u + 1, slab0 + rs, lane, wb[rs]);
-        lookup_unit<MU, NB, HALF, BT>(cur, off, acc[rs]);
+    constexpr int P = 32 / NB;
+    build_unit<MU, HALF, BT>(sbase, warp, lane);
+    if (tid < Geom<MU, BT>::kSlots && u + 1 < u_end) {
+        store_products<MU, BT>(sbase, HALF ^ 1, tid, pp.c1, pp.x1);
+        pp.c1 = pp.c2;
+        slot_x<BT>(a, b0, pp.col2, pp.x1);
+        if (u + 3 < u_end) {
+            const SlotStatic st = slot_static<MU, NB0, NB1>(a, u + 3, tid);
+            pp.c2 = st.c;
+            pp.col2 = st.col;
+        }
     }
+    float rsc[kSlabsPerWarp][NB];
     if (br.rgroup > 0) {
-        // block-wise row scales: the unit lies in one column block
-        constexpr int P = 32 / NB;
         const int g = (int)(((int64_t)ul * P * MU) / br.rgroup);
 #pragma unroll
         for (int rs = 0; rs < kSlabsPerWarp; ++rs) {
@@ -267,51 +414,65 @@ __device__ __forceinline__ void unit_step(const KernelArgs& a, int u, int u_end,
 #pragma unroll
             for (int ai = 0; ai < NB; ++ai) {
                 const int k = (ai + lane / P) % NB;
-                const float sc = i < a.M ? __half2float(br.r[((int64_t)k * br.ngroups + g) * a.M + i]) : 0.f;
-#pragma unroll
-                for (int b = 0; b < BT; ++b) {
-                    tot[rs][b] = fmaf(sc, acc[rs][b][ai], tot[rs][b]);
-                    acc[rs][b][ai] = 0.f;
-                }
+                rsc[rs][ai] = i < a.M ? __half2float(br.r[((int64_t)k * br.ngroups + g) * a.M + i]) : 0.f;
             }
         }
     }
+    __syncthreads();
+#pragma unroll
+    for (int rs = 0; rs < kSlabsPerWarp; ++rs) {
+        uint4 cur[Geom<MU, BT>::kVecs];
+#pragma unroll
+        for (int h = 0; h < Geom<MU, BT>::kVecs; ++h) cur[h] = wb.w[HALF][rs][h];
+        if (u + 2 < u_end) load_unit_slab<MU, BT>(a, u + 2, slab0 + rs, lane, wb.w[HALF][rs]);
+        lookup_unit<MU, NB, HALF, BT>(cur, off, sbase, acc[rs]);
+    }
+    if (br.rgroup > 0) {
+        // block-wise row scales: the unit lies in one column block
+#pragma unroll
+        for (int rs = 0; rs < kSlabsPerWarp; ++rs)
+#pragma unroll
+            for (int ai = 0; ai < NB; ++ai)
+#pragma unroll
+                for (int b = 0; b < BT; ++b) {
+                    tot[rs][b] = fmaf(rsc[rs][ai], acc[rs][b][ai], tot[rs][b]);
+                    acc[rs][b][ai] = 0.f;
+                }
+    }
 }
 
-template <int MU, int BR, int NB, int BT>
+template <int MU, int BR, int NB, int BT, int NB0, int NB1>
 __device__ __forceinline__ void run_branch(const KernelArgs& a, int u_lo, int u_hi, int u_end, int& v, int b0,
-                                           int slab0, int warp, int lane,
-                                           uint4 (&wb)[kSlabsPerWarp][Geom<MU>::kVecs],
+                                           int slab0, int warp, int lane, int tid, uint32_t sbase,
+                                           ProductPipe<BT>& pp, WeightRegs<MU, BT>& wb,
                                            float (&acc)[kSlabsPerWarp][BT][NB],
                                            float (&tot)[kSlabsPerWarp][BT]) {
     if (u_lo >= u_hi) return;
     Offsets<MU> off;
-    off.template make<NB>(lane);
+    off.template load<NB>(lane);
     const int ubase = BR ? a.br[0].units : 0;
     for (int u = u_lo; u < u_hi; ++u, ++v) {
         if (v & 1)
-            unit_step<MU, BR, NB, 1, BT>(a, u, u_end, u - ubase, b0, slab0, warp, lane, off, wb, acc, tot);
+            unit_step<MU, BR, NB, 1, BT, NB0, NB1>(a, u, u_end, u - ubase, b0, slab0, warp, lane, tid, sbase, off, pp,
+                                                   wb, acc, tot);
         else
-            unit_step<MU, BR, NB, 0, BT>(a, u, u_end, u - ubase, b0, slab0, warp, lane, off, wb, acc, tot);
+            unit_step<MU, BR, NB, 0, BT, NB0, NB1>(a, u, u_end, u - ubase, b0, slab0, warp, lane, tid, sbase, off, pp,
+                                                   wb, acc, tot);
     }
 }
 
-// Row-scale epilogue of one branch with per-row scales.
-template <int NB, int BT>
-__device__ __forceinline__ void apply_row_scales(const KernelArgs& a, const BranchArgs& br, int slab0, int lane,
-                                                 const float (&acc)[kSlabsPerWarp][BT][NB],
-                                                 float (&tot)[kSlabsPerWarp][BT]) {
+// Per-row scales of the lane's rows for one branch: sc[rs][a] = r_{k(a)}[row].
+template <int NB>
+__device__ __forceinline__ void fetch_row_scales(const KernelArgs& a, const BranchArgs& br, int slab0, int lane,
+                                                 float (&sc)[kSlabsPerWarp][NB]) {
     constexpr int P = 32 / NB;
 #pragma unroll
     for (int rs = 0; rs < kSlabsPerWarp; ++rs) {
         const int i = (slab0 + rs) * kLanes + lane;
-        if (i >= a.M) continue;
 #pragma unroll
         for (int ai = 0; ai < NB; ++ai) {
             const int k = (ai + lane / P) % NB;
-            const float sc = __half2float(br.r[(int64_t)k * a.M + i]);
-#pragma unroll
-            for (int b = 0; b < BT; ++b) tot[rs][b] = fmaf(sc, acc[rs][b][ai], tot[rs][b]);
+            sc[rs][ai] = (i < a.M && br.rgroup == 0 && br.units > 0) ? __half2float(br.r[(int64_t)k * a.M + i]) : 0.f;
         }
     }
 }
@@ -327,35 +488,83 @@ __device__ __forceinline__ void store_y(const KernelArgs& a, int b, int i, float
     }
 }
 
-template <int MU, int NB0, int NB1, int BT, int MINB>
-__global__ void __launch_bounds__(kThreads, MINB) fluxbin_lut_kernel(const KernelArgs a) {
+// Up to two CTAs per SM when one batch row is resident (their table builds
+// then overlap each other's lookups); larger batch tiles run one CTA per SM
+// with up to 255 registers a thread.
+template <int BT>
+constexpr int min_blocks() { return BT == 1 ? 2 : 1; }
+
+template <int MU, int NB0, int NB1, int BT>
+__global__ void __launch_bounds__(kThreads, min_blocks<BT>()) fluxbin_lut_kernel(const KernelArgs a) {
+    using G = Geom<MU, BT>;
     constexpr int NB1E = NB1 > 0 ? NB1 : 1;
     const int tid = threadIdx.x, warp = tid / kLanes, lane = tid % kLanes;
-    const int bc = blockIdx.x % a.n_bc;
-    const int ks = (blockIdx.x / a.n_bc) % a.n_ks;
-    const int rg = blockIdx.x / (a.n_bc * a.n_ks);
+    const int ks = blockIdx.x % a.n_ks;
+    const int bc = (blockIdx.x / a.n_ks) % a.n_bc;
+    const int rg = blockIdx.x / (a.n_ks * a.n_bc);
     const int b0 = bc * BT;
     const int slab0 = rg * kSlabsPerCta + warp * kSlabsPerWarp;
     const int U0 = a.br[0].units;
     const int U = U0 + (NB1 > 0 ? a.br[1].units : 0);
     const int u_begin = (int)(((int64_t)ks * U) / a.n_ks);
     const int u_end = (int)(((int64_t)(ks + 1) * U) / a.n_ks);
+    const uint32_t sbase = smem_base();
 
     // Let the next kernel on the stream start its own prologue.
     asm volatile("griddepcontrol.launch_dependents;");
 
-    uint4 wb[kSlabsPerWarp][Geom<MU>::kVecs];
+    WeightRegs<MU, BT> wb;
+    float sc0[kSlabsPerWarp][NB0], sc1[kSlabsPerWarp][NB1E];
+    SlotStatic st0{0.f, -1}, st1{0.f, -1}, st2{0.f, -1};
+    const bool slot_owner = tid < G::kSlots;
     const bool early = (a.flags & kFlagEarlyWeights) != 0;
-    if (early && u_begin < u_end) {
+    auto fetch_layer = [&]() {
 #pragma unroll
-        for (int rs = 0; rs < kSlabsPerWarp; ++rs) load_unit_slab<MU>(a, u_begin, slab0 + rs, lane, wb[rs]);
-    }
+        for (int d = 0; d < 2; ++d)
+            if (u_begin + d < u_end) {
+#pragma unroll
+                for (int rs = 0; rs < kSlabsPerWarp; ++rs)
+                    load_unit_slab<MU, BT>(a, u_begin + d, slab0 + rs, lane, wb.w[d][rs]);
+            }
+        if (tid < kSlabsPerCta && u_begin + 2 < u_end) {
+            // the rest of this CTA's packed words: one contiguous run per slab and branch
+            const int sl = rg * kSlabsPerCta + tid;
+            if (sl < a.Ms) {
+                const int g_lo = u_begin + 2, g_hi = min(u_end, U0);
+                if (g_lo < g_hi)
+                    prefetch_l2(a.br[0].words + ((int64_t)sl * U0 + g_lo) * (8 * MU), (uint32_t)(g_hi - g_lo) * 128u * MU);
+                if constexpr (NB1 > 0) {
+                    const int s_lo = max(u_begin + 2, U0) - U0, s_hi = u_end - U0;
+                    if (s_lo < s_hi)
+                        prefetch_l2(a.br[1].words + ((int64_t)sl * a.br[1].units + s_lo) * (8 * MU),
+                                    (uint32_t)(s_hi - s_lo) * 128u * MU);
+                }
+            }
+        }
+        fetch_row_scales<NB0>(a, a.br[0], slab0, lane, sc0);
+        if constexpr (NB1 > 0) fetch_row_scales<NB1>(a, a.br[1], slab0, lane, sc1);
+        if (slot_owner) {
+            if (u_begin < u_end) st0 = slot_static<MU, NB0, NB1>(a, u_begin, tid);
+            if (u_begin + 1 < u_end) st1 = slot_static<MU, NB0, NB1>(a, u_begin + 1, tid);
+            if (u_begin + 2 < u_end) st2 = slot_static<MU, NB0, NB1>(a, u_begin + 2, tid);
+        }
+    };
+    if (early) fetch_layer();
     // Everything below may read what the preceding kernel wrote.
     asm volatile("griddepcontrol.wait;" ::: "memory");
-    if (!early && u_begin < u_end) {
-#pragma unroll
-        for (int rs = 0; rs < kSlabsPerWarp; ++rs) load_unit_slab<MU>(a, u_begin, slab0 + rs, lane, wb[rs]);
+    if (!early) fetch_layer();
+
+    ProductPipe<BT> pp;
+    if (slot_owner) {
+        __half x0[BT];
+        slot_x<BT>(a, b0, st0.col, x0);
+        slot_x<BT>(a, b0, st1.col, pp.x1);
+        if (u_begin < u_end) store_products<MU, BT>(sbase, 0, tid, st0.c, x0);
+        pp.c1 = st1.c;
+        pp.c2 = st2.c;
+        pp.col2 = st2.col;
     }
+    __syncthreads();
 
     float acc0[kSlabsPerWarp][BT][NB0];
     float acc1[kSlabsPerWarp][BT][NB1E];
@@ -372,18 +581,26 @@ __global__ void __launch_bounds__(kThreads, MINB) fluxbin_lut_kernel(const Kerne
         }
 
     int v = 0;
-    run_branch<MU, 0, NB0, BT>(a, u_begin, min(u_end, U0), u_end, v, b0, slab0, warp, lane, wb, acc0, tot);
+    run_branch<MU, 0, NB0, BT, NB0, NB1>(a, u_begin, min(u_end, U0), u_end, v, b0, slab0, warp, lane, tid, sbase,
+                                         pp, wb, acc0, tot);
     if constexpr (NB1 > 0)
-        run_branch<MU, 1, NB1, BT>(a, max(u_begin, U0), u_end, u_end, v, b0, slab0, warp, lane, wb, acc1, tot);
+        run_branch<MU, 1, NB1, BT, NB0, NB1>(a, max(u_begin, U0), u_end, u_end, v, b0, slab0, warp, lane, tid, sbase,
+                                             pp, wb, acc1, tot);
 
     // Row scales (per-row case; the block-wise case was applied per unit).
-    if (a.br[0].rgroup == 0 && u_begin < min(u_end, U0))
-        apply_row_scales<NB0, BT>(a, a.br[0], slab0, lane, acc0, tot);
-    if constexpr (NB1 > 0) {
-        if (a.br[1].rgroup == 0 && max(u_begin, U0) < u_end)
-            apply_row_scales<NB1, BT>(a, a.br[1], slab0, lane, acc1, tot);
-    }
+#pragma unroll
+    for (int rs = 0; rs < kSlabsPerWarp; ++rs)
+#pragma unroll
+        for (int b = 0; b < BT; ++b) {
+#pragma unroll
+            for (int q = 0; q < NB0; ++q) tot[rs][b] = fmaf(sc0[rs][q], acc0[rs][b][q], tot[rs][b]);
+            if constexpr (NB1 > 0) {
+#pragma unroll
+                for (int q = 0; q < NB1; ++q) tot[rs][b] = fmaf(sc1[rs][q], acc1[rs][b][q], tot[rs][b]);
+            }
+        }
 
+    const int row0 = rg * kRowsPerCta;
     if (a.n_ks == 1) {
 #pragma unroll
         for (int rs = 0; rs < kSlabsPerWarp; ++rs) {
@@ -396,7 +613,38 @@ __global__ void __launch_bounds__(kThreads, MINB) fluxbin_lut_kernel(const Kerne
         return;
     }
 
-    // Split-K: add this CTA's partial sums; the last CTA of the group finishes.
+    if (a.cluster) {
+        // Split-K reduction inside the cluster: every CTA parks its partials in
+        // its own shared memory; CTA r then sums slice r of the rows over all
+        // CTAs in rank order and writes y.
+        const uint32_t red = sbase + G::kRedOff;
+#pragma unroll
+        for (int rs = 0; rs < kSlabsPerWarp; ++rs) {
+            const int lr = (warp * kSlabsPerWarp + rs) * kLanes + lane;
+#pragma unroll
+            for (int b = 0; b < BT; ++b) sts_f32(red + (uint32_t)(b * kRowsPerCta + lr) * 4u, tot[rs][b]);
+        }
+        cluster_sync_all();
+        const int C = a.n_ks;
+        const int rank = (int)cluster_rank();
+        const int chunk = (kRowsPerCta + C - 1) / C;
+        for (int e = tid; e < BT * chunk; e += kThreads) {
+            const int b = e / chunk, lr = rank * chunk + e % chunk;
+            if (lr >= kRowsPerCta) continue;
+            const int i = row0 + lr;
+            if (i >= a.M || b0 + b >= a.B) continue;
+            const uint32_t off = red + (uint32_t)(b * kRowsPerCta + lr) * 4u;
+            float s = 0.f;
+            for (int c = 0; c < C; ++c) s += ld_dsmem_f32(off, (uint32_t)c);
+            store_y(a, b0 + b, i, s);
+        }
+        // keep every CTA's shared memory alive until all reads are done
+        cluster_sync_all();
+        return;
+    }
+
+    // Split-K through the workspace: add this CTA's partials; the last CTA of
+    // the row group to arrive finishes the sum, writes y and re-zeroes it.
 #pragma unroll
     for (int rs = 0; rs < kSlabsPerWarp; ++rs) {
         const int i = (slab0 + rs) * kLanes + lane;
@@ -413,7 +661,6 @@ __global__ void __launch_bounds__(kThreads, MINB) fluxbin_lut_kernel(const Kerne
     __syncthreads();
     if (!s_last) return;
     __threadfence();
-    const int row0 = rg * kRowsPerCta;
     for (int e = tid; e < kRowsPerCta * BT; e += kThreads) {
         const int b = e / kRowsPerCta, i = row0 + e % kRowsPerCta;
         if (i >= a.M || b0 + b >= a.B) continue;

@@ -6,9 +6,9 @@
 #include <stdint.h>
 
 #if defined(__CUDACC__)
-#define FB_HD __host__ __device__ __forceinline__
+#define FB_HD __host__ __device__ constexpr
 #else
-#define FB_HD inline
+#define FB_HD constexpr
 #endif
 
 namespace fluxbin {
@@ -16,9 +16,10 @@ namespace fluxbin {
 constexpr int kLanes = 32;          // rows per slab = lanes per warp = shared-memory banks
 constexpr int kWarps = 8;           // warps per CTA
 constexpr int kThreads = kWarps * kLanes;
-constexpr int kSlabsPerWarp = 4;    // row slabs a warp keeps accumulators for
+constexpr int kSlabsPerWarp = 2;    // row slabs a warp keeps accumulators for
 constexpr int kSlabsPerCta = kWarps * kSlabsPerWarp;
-constexpr int kRowsPerCta = kSlabsPerCta * kLanes;  // 1024
+constexpr int kRowsPerCta = kSlabsPerCta * kLanes;  // 512
+constexpr int kMaxCluster = 16;     // CTAs that reduce their split-K partials through DSMEM
 constexpr int kMaxBatch = 16;
 
 // Sub-vectors of one base inside a unit.

@@ -89,6 +89,9 @@ CASES = [
     (spec(64, 2048, 2, 0, 0, 8, G=128), 1),  # block-wise row scales
     (spec(1100, 1024, 2, 1, 64, 4, G=128), 3),
     (spec(1100, 1024, 1, 0, 0, 8, G=256), 2),
+    (spec(256, 65536, 2, 1, 300, 8), 1),     # split wider than a cluster: workspace path
+    (spec(100, 30000, 1, 2, 500, 4), 3),
+    (spec(4096, 4096, 2, 1, 205, 8), 2),
 ]
 
 
@@ -175,8 +178,9 @@ def test_noop_and_errors_on_device():
     x = torch.zeros((0, sp.N), dtype=torch.float16, device="cuda")
     y = torch.zeros((0, sp.M), dtype=torch.float32, device="cuda")
     d.linear(x, y, fluxbin.FLAG_Y_FP32, None)   # B = 0: nothing to do
-    # a layer that needs split-K refuses to run without a workspace
-    big = spec(4096, 4096, 2, 1, 205, 8)
+    # a layer whose reduction is split wider than a cluster refuses to run
+    # without a workspace (few rows, very long rows)
+    big = spec(256, 65536, 2, 1, 205, 8)
     lb = fluxbin.DeviceLayer.from_host(synth.make_layer(big, [97]))
     xb = torch.zeros((1, big.N), dtype=torch.float16, device="cuda")
     yb = torch.zeros((1, big.M), dtype=torch.float32, device="cuda")

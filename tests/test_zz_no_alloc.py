@@ -40,6 +40,7 @@ def close(got, ref, layer, x):
     (synth.layer_7b_proj(), 1),
     (LayerSpec("ragged", 2100, 777, 2, 1, 40, 8), 3),
     (LayerSpec("mu4", 1500, 1030, 2, 2, 60, 4), 5),
+    (LayerSpec("wide", 256, 65536, 2, 1, 300, 8), 2),   # reduction through the scratch
 ])
 def test_static_scratch_matches_workspace_entry_point(sp, B):
     if not torch.cuda.is_available():
