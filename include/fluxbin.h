@@ -125,6 +125,10 @@ typedef struct fluxbin_layer_desc {
 /* Human-readable name of a status code (static storage, never NULL). */
 const char* fluxbin_status_string(int status);
 
+/* Name and description of the last CUDA failure (FLUXBIN_ERR_CUDA) seen by a
+ * call on this host thread; "" if none.  Thread-local storage, never NULL. */
+const char* fluxbin_last_error(void);
+
 /* Library version: major*10000 + minor*100 + patch. */
 int fluxbin_version(void);
 

@@ -3,6 +3,7 @@
 // are in include/fluxbin.h.
 #include <cuda_runtime.h>
 
+#include <cstdio>
 #include <mutex>
 #include <unordered_map>
 
@@ -16,6 +17,15 @@ KernelFn select_kernel_mu8(int nb0, int nb1, int bt);
 KernelFn select_kernel_mu4(int nb0, int nb1, int bt);
 
 namespace {
+
+thread_local char g_last_error[256] = "";
+
+// Records a failed CUDA call for fluxbin_last_error() and clears the error state.
+int cuda_fail(cudaError_t e) {
+    snprintf(g_last_error, sizeof(g_last_error), "%s: %s", cudaGetErrorName(e), cudaGetErrorString(e));
+    (void)cudaGetLastError();
+    return FLUXBIN_ERR_CUDA;
+}
 
 // Batch rows whose tables a CTA keeps resident (the rest go to other CTAs).
 int batch_tile(int mu, int B) {
@@ -70,13 +80,15 @@ int func_info(KernelFn fn, int dev, int mu, int bt, const DeviceInfo& di, FuncIn
     }
     FuncInfo fi;
     const size_t smem_max = table_smem_bytes(mu, bt) + red_smem_bytes(bt);
-    if ((size_t)di.max_smem < smem_max) return FLUXBIN_ERR_SMEM_BUDGET;
-    if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_max) != cudaSuccess ||
-        cudaFuncSetAttribute(fn, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess ||
-        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&fi.blocks_per_sm, fn, kThreads, smem_max) != cudaSuccess) {
-        (void)cudaGetLastError();
-        return FLUXBIN_ERR_CUDA;
-    }
+    cudaFuncAttributes fa;
+    cudaError_t e = cudaFuncGetAttributes(&fa, fn);
+    if (e != cudaSuccess) return cuda_fail(e);
+    // the dynamic allocation shares the per-block limit with the static one
+    if ((size_t)di.max_smem < smem_max + fa.sharedSizeBytes) return FLUXBIN_ERR_SMEM_BUDGET;
+    if ((e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_max)) != cudaSuccess ||
+        (e = cudaFuncSetAttribute(fn, cudaFuncAttributeNonPortableClusterSizeAllowed, 1)) != cudaSuccess ||
+        (e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&fi.blocks_per_sm, fn, kThreads, smem_max)) != cudaSuccess)
+        return cuda_fail(e);
     if (fi.blocks_per_sm < 1) return FLUXBIN_ERR_SMEM_BUDGET;
     g_func.emplace(key, fi);
     *out = fi;
@@ -127,23 +139,17 @@ struct Plan {
 
 // Row groups of 512 rows times batch chunks fix the number of CTA groups; the
 // units are split over up to 16 CTAs per group forming a cluster whose
-// partials are reduced in DSMEM.  A layer whose packed words come to at most
-// kSmallLayerBytesPerSm per SM gets at most one CTA per SM, so that the CTAs
-// of the next call on the stream fit beside them and fetch their own words
-// while this call finishes (programmatic dependent launch); larger layers
-// fill every CTA slot.  Every cluster must be resident at once.  When that
+// partials are reduced in DSMEM, choosing the widest split for which every
+// cluster is resident at once, up to one CTA per CTA slot of the GPU (two per
+// SM: one CTA's table build then overlaps the other's lookups).  When that
 // leaves most SMs idle (few rows, long rows) the units are split as widely
 // as the SMs allow and reduced through the workspace.
-constexpr int64_t kSmallLayerBytesPerSm = 96 * 1024;
-
 Plan make_plan(KernelFn fn, int dev, int mu, int bt, int64_t Ms, int64_t U, int n_bc, const DeviceInfo& di,
                const FuncInfo& fi) {
     Plan p;
     p.n_rg = (int)((Ms + kSlabsPerCta - 1) / kSlabsPerCta);
     const int64_t groups = (int64_t)p.n_rg * n_bc;
-    const int64_t layer_bytes = Ms * U * 128 * mu;
-    const bool small = layer_bytes <= kSmallLayerBytesPerSm * di.sm_count;
-    const int64_t slots = (int64_t)di.sm_count * (small ? 1 : fi.blocks_per_sm);
+    const int64_t slots = (int64_t)di.sm_count * fi.blocks_per_sm;
     int64_t want = slots / groups;
     if (want > U) want = U;
     if (want > kMaxCluster) want = kMaxCluster;
@@ -256,10 +262,8 @@ int run(int32_t M, int32_t N, int mu, const BranchIn& g, const BranchIn* s, cons
         attr[1].val.clusterDim.z = 1;
         cfg.numAttrs = 2;
     }
-    if (cudaLaunchKernelEx(&cfg, fn, a) != cudaSuccess) {
-        (void)cudaGetLastError();
-        return FLUXBIN_ERR_CUDA;
-    }
+    const cudaError_t le = cudaLaunchKernelEx(&cfg, fn, a);
+    if (le != cudaSuccess) return cuda_fail(le);
     return FLUXBIN_OK;
 }
 
@@ -269,6 +273,8 @@ int run(int32_t M, int32_t N, int mu, const BranchIn& g, const BranchIn* s, cons
 using namespace fluxbin;
 
 extern "C" {
+
+const char* fluxbin_last_error(void) { return g_last_error; }
 
 int fluxbin_lut_gemv(int32_t M, int32_t N, int32_t ncols, int32_t nbases, int32_t mu, int32_t row_scale_group,
                      const uint32_t* d_words, const uint16_t* d_r, const uint16_t* d_c, const int32_t* d_gather,

@@ -170,11 +170,6 @@ __device__ __forceinline__ float sum_f32x2(uint64_t x) {
     return lo + hi;
 }
 
-// Ask the L2 to fetch [p, p + bytes) from HBM (bytes a multiple of 16).
-__device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
-    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
-}
-
 __device__ __forceinline__ void red_add_f32(float* p, float v) {
     asm volatile("red.global.add.f32 [%0], %1;" ::"l"(p), "f"(v) : "memory");
 }
@@ -526,21 +521,6 @@ __global__ void __launch_bounds__(kThreads, min_blocks<BT>()) fluxbin_lut_kernel
                 for (int rs = 0; rs < kSlabsPerWarp; ++rs)
                     load_unit_slab<MU, BT>(a, u_begin + d, slab0 + rs, lane, wb.w[d][rs]);
             }
-        if (tid < kSlabsPerCta && u_begin + 2 < u_end) {
-            // the rest of this CTA's packed words: one contiguous run per slab and branch
-            const int sl = rg * kSlabsPerCta + tid;
-            if (sl < a.Ms) {
-                const int g_lo = u_begin + 2, g_hi = min(u_end, U0);
-                if (g_lo < g_hi)
-                    prefetch_l2(a.br[0].words + ((int64_t)sl * U0 + g_lo) * (8 * MU), (uint32_t)(g_hi - g_lo) * 128u * MU);
-                if constexpr (NB1 > 0) {
-                    const int s_lo = max(u_begin + 2, U0) - U0, s_hi = u_end - U0;
-                    if (s_lo < s_hi)
-                        prefetch_l2(a.br[1].words + ((int64_t)sl * a.br[1].units + s_lo) * (8 * MU),
-                                    (uint32_t)(s_hi - s_lo) * 128u * MU);
-                }
-            }
-        }
         fetch_row_scales<NB0>(a, a.br[0], slab0, lane, sc0);
         if constexpr (NB1 > 0) fetch_row_scales<NB1>(a, a.br[1], slab0, lane, sc1);
         if (slot_owner) {

@@ -35,7 +35,8 @@ class FluxbinLibraryMissing(ImportError):
 class FluxbinError(RuntimeError):
     def __init__(self, status: int, where: str):
         self.status = status
-        super().__init__(f"{where}: {STATUS.get(status, status)} ({fluxbin_status_string(status)})")
+        detail = f"; {fluxbin_last_error()}" if status == -7 else ""
+        super().__init__(f"{where}: {STATUS.get(status, status)} ({fluxbin_status_string(status)}{detail})")
 
 
 class LayerDesc(ctypes.Structure):
@@ -65,6 +66,7 @@ def lib():
             L.fluxbin_status_string.argtypes = [ctypes.c_int]
             L.fluxbin_status_string.restype = ctypes.c_char_p
             L.fluxbin_version.restype = ctypes.c_int
+            L.fluxbin_last_error.restype = ctypes.c_char_p
             L.fluxbin_packed_sizes.argtypes = [P, ctypes.POINTER(sz), ctypes.POINTER(sz)]
             L.fluxbin_pack.argtypes = [P, P, P, P, P, P]
             L.fluxbin_workspace_bytes.argtypes = [i32, i32, ctypes.POINTER(sz)]
@@ -85,6 +87,10 @@ def _check(st: int, where: str) -> None:
 
 def fluxbin_status_string(status: int) -> str:
     return lib().fluxbin_status_string(int(status)).decode()
+
+
+def fluxbin_last_error() -> str:
+    return lib().fluxbin_last_error().decode()
 
 
 def fluxbin_version() -> int:
