@@ -57,6 +57,14 @@
  *   word = (s*U + u)*32*mu + ((pos / 128)*32 + L)*4 + (pos / 32) % 4
  *   bit  = pos % 32
  *
+ * Grouped order.  A salient branch whose row scales change every Gs salient
+ * columns with Gs a multiple of mu and gsv = Gs/mu in {1, 2, 4} dividing P
+ * (sal_scale_group smaller than a unit) uses instead, with KG = 32/gsv and
+ * NG = P/gsv, lane L = gsv*m + sg (m = L/gsv, sg = L%gsv):
+ *   kg = k*NG + j/gsv,  a = (kg - m) mod KG,  q = a*gsv + ((j % gsv) xor sg)
+ * so that the steps a*gsv .. a*gsv+gsv-1 of a lane cover one whole (base,
+ * scale group) and the lane can apply that group's row scale once.
+ *
  * Reading: lane L of a warp owns row 32*s + L.  Over its 32 steps q it visits
  * the unit's 32 (base, sub-vector) tables in the order
  *   base k = (q/P + L/P) mod nb, sub-vector j = (L + q) mod P,
@@ -73,7 +81,8 @@
  *   r  [Kb][M]            (row_scale_group == 0: one per row)
  *   r  [Kb][ceil(N/G)][M] (row_scale_group == G > 0: one per row per G-column
  *                          block, Appendix C.2 "block-wise row scales")
- *   rs [Ks][M] or [Ks][ceil(n_sal/Gs)][M]       (sal_scale_group == Gs)
+ *   rs [Ks][M] or [Ks][ceil(n_sal/Gs)][M]       (sal_scale_group == Gs: a multiple of
+ *                                               the unit width, or Gs = gsv*mu as above)
  *   x  [B][N], y [B][M] (row-major; y fp16 or fp32)
  *   idx[n_sal] int32, strictly increasing, < N  (the salient column set S)
  */
@@ -93,7 +102,8 @@ typedef enum fluxbin_status {
     FLUXBIN_ERR_BAD_SHAPE = -2,    /* negative or inconsistent sizes, bad salient index list */
     FLUXBIN_ERR_MISALIGNED = -3,   /* a device pointer lacks the alignment stated below */
     FLUXBIN_ERR_UNSUPPORTED = -4,  /* mu not in {4,8}; Kb not in {1,2,4}; Ks not in {0,1,2,4};
-                                      B > 16; a scale block that does not hold whole units */
+                                      B > 16; a row-scale block that does not hold whole units
+                                      (salient: nor 1, 2 or 4 whole sub-vectors) */
     FLUXBIN_ERR_SMEM_BUDGET = -5,  /* the tables for this shape do not fit in shared memory */
     FLUXBIN_ERR_WORKSPACE = -6,    /* workspace missing or smaller than fluxbin_workspace_bytes() */
     FLUXBIN_ERR_CUDA = -7,         /* a CUDA runtime call or the kernel launch failed */
@@ -109,7 +119,9 @@ typedef struct fluxbin_layer_desc {
     int32_t n_sal;            /* salient columns, 0 <= n_sal <= N (0 when Ks == 0) */
     int32_t mu;               /* LUT sub-vector length: 4 or 8 */
     int32_t row_scale_group;  /* 0: one row scale per row; G > 0: one per row per G columns */
-    int32_t sal_scale_group;  /* 0: one salient row scale per row; Gs > 0: one per Gs salient columns */
+    int32_t sal_scale_group;  /* 0: one salient row scale per row; Gs > 0: one per Gs salient columns
+                                 (a multiple of the unit width (32/Ks)*mu, or mu, 2*mu or 4*mu
+                                 dividing it: grouped visit order) */
 } fluxbin_layer_desc;
 
 /* Flags for the device entry points. */

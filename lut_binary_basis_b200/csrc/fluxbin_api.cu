@@ -13,8 +13,8 @@
 namespace fluxbin {
 
 using KernelFn = void (*)(KernelArgs);
-KernelFn select_kernel_mu8(int nb0, int nb1, int bt);
-KernelFn select_kernel_mu4(int nb0, int nb1, int bt);
+KernelFn select_kernel_mu8(int nb0, int nb1, int bt, int gs1);
+KernelFn select_kernel_mu4(int nb0, int nb1, int bt, int gs1);
 
 namespace {
 
@@ -37,6 +37,9 @@ int batch_tile(int mu, int B) {
 size_t table_smem_bytes(int mu, int bt) {
     return (size_t)bt * ((size_t)1 << mu) * 256u + 2u * (size_t)bt * 32u * (size_t)mu * sizeof(float);
 }
+// Staged row scales of a grouped salient branch: two parities of one fp16
+// per slot (32/gs1 of them) and row of the CTA.
+size_t scale_smem_bytes(int gs1) { return gs1 > 0 ? 2u * (32u / (size_t)gs1) * kRowsPerCta * 2u : 0u; }
 // Cluster reduction buffer: one fp32 partial per row of the CTA and batch row.
 size_t red_smem_bytes(int bt) { return (size_t)bt * kRowsPerCta * sizeof(float); }
 
@@ -71,7 +74,7 @@ int device_info(int dev, DeviceInfo* out) {
 
 // Per-function, per-device set-up: opt in to the dynamic shared memory of the
 // largest launch and to non-portable cluster sizes; occupancy.
-int func_info(KernelFn fn, int dev, int mu, int bt, const DeviceInfo& di, FuncInfo* out) {
+int func_info(KernelFn fn, int dev, int mu, int bt, int gs1, const DeviceInfo& di, FuncInfo* out) {
     const uint64_t key = (reinterpret_cast<uint64_t>(fn) << 8) ^ (uint64_t)dev;
     auto it = g_func.find(key);
     if (it != g_func.end()) {
@@ -79,7 +82,7 @@ int func_info(KernelFn fn, int dev, int mu, int bt, const DeviceInfo& di, FuncIn
         return FLUXBIN_OK;
     }
     FuncInfo fi;
-    const size_t smem_max = table_smem_bytes(mu, bt) + red_smem_bytes(bt);
+    const size_t smem_max = table_smem_bytes(mu, bt) + red_smem_bytes(bt) + scale_smem_bytes(gs1);
     cudaFuncAttributes fa;
     cudaError_t e = cudaFuncGetAttributes(&fa, fn);
     if (e != cudaSuccess) return cuda_fail(e);
@@ -144,8 +147,8 @@ struct Plan {
 // SM: one CTA's table build then overlaps the other's lookups).  When that
 // leaves most SMs idle (few rows, long rows) the units are split as widely
 // as the SMs allow and reduced through the workspace.
-Plan make_plan(KernelFn fn, int dev, int mu, int bt, int64_t Ms, int64_t U, int n_bc, const DeviceInfo& di,
-               const FuncInfo& fi) {
+Plan make_plan(KernelFn fn, int dev, int mu, int bt, int gs1, int64_t Ms, int64_t U, int n_bc,
+               const DeviceInfo& di, const FuncInfo& fi) {
     Plan p;
     p.n_rg = (int)((Ms + kSlabsPerCta - 1) / kSlabsPerCta);
     const int64_t groups = (int64_t)p.n_rg * n_bc;
@@ -153,7 +156,7 @@ Plan make_plan(KernelFn fn, int dev, int mu, int bt, int64_t Ms, int64_t U, int 
     int64_t want = slots / groups;
     if (want > U) want = U;
     if (want > kMaxCluster) want = kMaxCluster;
-    const size_t smem = table_smem_bytes(mu, bt) + red_smem_bytes(bt);
+    const size_t smem = table_smem_bytes(mu, bt) + red_smem_bytes(bt) + scale_smem_bytes(gs1);
     for (int64_t ks = want; ks >= 2; --ks) {
         if (groups * ks * 2 < di.sm_count) break;  // too few CTAs: use the workspace instead
         if (max_active_clusters(fn, dev, (int)ks, smem) >= groups) {
@@ -191,8 +194,10 @@ int run(int32_t M, int32_t N, int mu, const BranchIn& g, const BranchIn* s, cons
         if (!aligned(b->r, 2) || !aligned(b->c, 2) || !aligned(b->gather, 4)) return FLUXBIN_ERR_MISALIGNED;
     }
     const int nb1 = (s && s->ncols > 0) ? s->nb : 0;
-    const int bt = batch_tile(mu, B);
-    KernelFn fn = mu == 8 ? select_kernel_mu8(g.nb, nb1, bt) : select_kernel_mu4(g.nb, nb1, bt);
+    // salient row scales finer than a unit: grouped visit order, one batch row per CTA
+    const int gs1 = (nb1 && s->rgroup > 0 && s->rgroup < unit_cols(nb1, mu)) ? s->rgroup / mu : 0;
+    const int bt = gs1 ? 1 : batch_tile(mu, B);
+    KernelFn fn = mu == 8 ? select_kernel_mu8(g.nb, nb1, bt, gs1) : select_kernel_mu4(g.nb, nb1, bt, gs1);
     if (!fn) return FLUXBIN_ERR_UNSUPPORTED;
 
     int dev = 0;
@@ -221,9 +226,9 @@ int run(int32_t M, int32_t N, int mu, const BranchIn& g, const BranchIn* s, cons
         std::lock_guard<std::mutex> lock(g_mu);
         int st = device_info(dev, &di);
         if (st != FLUXBIN_OK) return st;
-        st = func_info(fn, dev, mu, bt, di, &fi);
+        st = func_info(fn, dev, mu, bt, gs1, di, &fi);
         if (st != FLUXBIN_OK) return st;
-        plan = make_plan(fn, dev, mu, bt, a.Ms, U, n_bc, di, fi);
+        plan = make_plan(fn, dev, mu, bt, gs1, a.Ms, U, n_bc, di, fi);
     }
     a.x = reinterpret_cast<const __half*>(d_x);
     a.y = d_y;
@@ -248,7 +253,7 @@ int run(int32_t M, int32_t N, int mu, const BranchIn& g, const BranchIn* s, cons
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)((int64_t)a.n_rg * a.n_bc * a.n_ks));
     cfg.blockDim = dim3(kThreads);
-    cfg.dynamicSmemBytes = table_smem_bytes(mu, bt) + (plan.cluster ? red_smem_bytes(bt) : 0);
+    cfg.dynamicSmemBytes = table_smem_bytes(mu, bt) + red_smem_bytes(bt) + scale_smem_bytes(gs1);
     cfg.stream = static_cast<cudaStream_t>(stream);
     cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;

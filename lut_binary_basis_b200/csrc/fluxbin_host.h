@@ -14,6 +14,16 @@ inline bool valid_mu(int mu) { return mu == 4 || mu == 8; }
 
 inline bool has_salient(const fluxbin_layer_desc& d) { return d.Ks > 0 && d.n_sal > 0; }
 
+// Salient row-scale groups: whole units, or a power-of-two number of whole
+// sub-vectors (1, 2 or 4) that divides a unit (grouped visit order).
+inline bool valid_salient_group(int nb, int mu, int s) {
+    const int w = unit_cols(nb, mu);
+    if (s % w == 0) return true;
+    if (s % mu) return false;
+    const int g = s / mu;
+    return (g == 1 || g == 2 || g == 4) && w % s == 0;
+}
+
 // Checks the shape fields of a layer description.
 inline int validate_desc(const fluxbin_layer_desc* d) {
     if (!d) return FLUXBIN_ERR_INVALID_ARG;
@@ -26,7 +36,7 @@ inline int validate_desc(const fluxbin_layer_desc* d) {
     // block-wise row scales: a block must hold whole units, so that the scale
     // is constant across the unit a CTA accumulates before applying it
     if (d->row_scale_group > 0 && d->row_scale_group % unit_cols(d->Kb, d->mu)) return FLUXBIN_ERR_UNSUPPORTED;
-    if (has_salient(*d) && d->sal_scale_group > 0 && d->sal_scale_group % unit_cols(d->Ks, d->mu))
+    if (has_salient(*d) && d->sal_scale_group > 0 && !valid_salient_group(d->Ks, d->mu, d->sal_scale_group))
         return FLUXBIN_ERR_UNSUPPORTED;
     return FLUXBIN_OK;
 }

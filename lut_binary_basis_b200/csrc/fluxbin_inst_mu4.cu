@@ -6,15 +6,15 @@ namespace fluxbin {
 using KernelFn = void (*)(KernelArgs);
 
 namespace {
-template <int BT>
+template <int BT, int GS1>
 KernelFn pick(int nb0, int nb1) {
-#define FB_NB1(NB0)                                             \
-    switch (nb1) {                                              \
-        case 0: return &fluxbin_lut_kernel<4, NB0, 0, BT>;  \
-        case 1: return &fluxbin_lut_kernel<4, NB0, 1, BT>;  \
-        case 2: return &fluxbin_lut_kernel<4, NB0, 2, BT>;  \
-        case 4: return &fluxbin_lut_kernel<4, NB0, 4, BT>;  \
-        default: return nullptr;                                \
+#define FB_NB1(NB0)                                                        \
+    switch (nb1) {                                                         \
+        case 0: return GS1 ? nullptr : &fluxbin_lut_kernel<4, NB0, 0, BT, 0>; \
+        case 1: return &fluxbin_lut_kernel<4, NB0, 1, BT, GS1>;          \
+        case 2: return &fluxbin_lut_kernel<4, NB0, 2, BT, GS1>;          \
+        case 4: return &fluxbin_lut_kernel<4, NB0, 4, BT, GS1>;          \
+        default: return nullptr;                                           \
     }
     switch (nb0) {
         case 1: FB_NB1(1)
@@ -27,10 +27,19 @@ KernelFn pick(int nb0, int nb1) {
 }  // namespace
 
 // Tables of one batch row take 4 KiB; the batch tile is bounded by registers.
-KernelFn select_kernel_mu4(int nb0, int nb1, int bt) {
-    if (bt == 1) return pick<1>(nb0, nb1);
-    if (bt == 2) return pick<2>(nb0, nb1);
-    if (bt == 4) return pick<4>(nb0, nb1);
+// gs1 > 0: the salient branch has row scales per group of gs1 sub-vectors
+// (one batch row per CTA).
+KernelFn select_kernel_mu4(int nb0, int nb1, int bt, int gs1) {
+    if (gs1 > 0) {
+        if (bt != 1) return nullptr;
+        if (gs1 == 1) return pick<1, 1>(nb0, nb1);
+        if (gs1 == 2) return pick<1, 2>(nb0, nb1);
+        if (gs1 == 4) return pick<1, 4>(nb0, nb1);
+        return nullptr;
+    }
+    if (bt == 1) return pick<1, 0>(nb0, nb1);
+    if (bt == 2) return pick<2, 0>(nb0, nb1);
+    if (bt == 4) return pick<4, 0>(nb0, nb1);
     return nullptr;
 }
 

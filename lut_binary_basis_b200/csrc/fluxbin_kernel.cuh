@@ -43,6 +43,8 @@
 //           alternate halves: double buffering with one barrier per unit)
 //   vbuf    2 * BT * 32*mu floats: [parity][b][bank][t] activation products
 //   red     BT * 512 floats: partial sums for the cluster reduction
+//   scales  (grouped salient branch only) 2 * (32/gsv) * 512 fp16: the row
+//           scale each lane applies after each group, [parity][slot][row]
 #pragma once
 
 #include <cuda_fp16.h>
@@ -96,28 +98,37 @@ struct Geom {
     static constexpr int kVbufBytes = 2 * BT * kSlots * 4;
     static constexpr int kRedOff = kVbufOff + kVbufBytes;
     static constexpr int kRedBytes = BT * kRowsPerCta * 4;
+    static constexpr int kScaleOff = kRedOff + kRedBytes;  // grouped salient branch: staged scales
 };
 
 // Byte offsets (bank * 4) of the tables lane L visits at steps 3r, 3r+1, 3r+2,
-// packed into bytes 0..2 of word [nb index][r][L]; byte 3 is zero.
+// packed into bytes 0..2 of word [nb index][order][r][L]; byte 3 is zero.
+// Order 0 is the diagonal visit order, orders 1..3 the grouped order with
+// 1, 2 or 4 sub-vectors per row-scale group.
 struct OffsetTable {
-    uint32_t w[3][11][32];
+    uint32_t w[3][4][11][32];
 };
 constexpr OffsetTable make_offset_table() {
     OffsetTable t{};
     for (int nbi = 0; nbi < 3; ++nbi)
-        for (int r = 0; r < 11; ++r)
-            for (int L = 0; L < 32; ++L) {
-                uint32_t v = 0;
-                for (int m = 0; m < 3; ++m) {
-                    const int q = 3 * r + m;
-                    if (q < 32) v |= (uint32_t)(visit_bank(L, q, 1 << nbi) * 4) << (8 * m);
+        for (int o = 0; o < 4; ++o)
+            for (int r = 0; r < 11; ++r)
+                for (int L = 0; L < 32; ++L) {
+                    const int nb = 1 << nbi;
+                    const int gsv = o == 0 ? subvecs_per_unit(nb) : (1 << (o - 1));
+                    uint32_t v = 0;
+                    for (int m = 0; m < 3; ++m) {
+                        const int q = 3 * r + m;
+                        if (q < 32) v |= (uint32_t)(visit_bank(L, q, nb, gsv) * 4) << (8 * m);
+                    }
+                    t.w[nbi][o][r][L] = v;
                 }
-                t.w[nbi][r][L] = v;
-            }
     return t;
 }
 __device__ const OffsetTable kOffsetTable = make_offset_table();
+
+template <int GSV>
+constexpr int order_index() { return GSV == 0 ? 0 : (GSV == 1 ? 1 : (GSV == 2 ? 2 : 3)); }
 
 template <int NB>
 constexpr int nb_index() { return NB == 1 ? 0 : (NB == 2 ? 1 : 2); }
@@ -131,6 +142,13 @@ __device__ __forceinline__ uint4 ld_stream(const uint4* p) {
     asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
                  : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
     return v;
+}
+
+// Plain (compiler-scheduled) shared-memory access by byte offset from the
+// start of the dynamic allocation.
+template <typename T>
+__device__ __forceinline__ T& smem_at(uint32_t byte_off) {
+    return *reinterpret_cast<T*>(fb_smem + byte_off);
 }
 
 // Shared-memory access by 32-bit shared address (+ a constant byte offset).
@@ -196,10 +214,10 @@ __device__ __forceinline__ float ld_dsmem_f32(uint32_t local_smem_addr, uint32_t
 template <int MU>
 struct Offsets {
     uint32_t o[11];
-    template <int NB>
+    template <int NB, int GSV>
     __device__ __forceinline__ void load(int lane) {
 #pragma unroll
-        for (int r = 0; r < 11; ++r) o[r] = __ldg(&kOffsetTable.w[nb_index<NB>()][r][lane]);
+        for (int r = 0; r < 11; ++r) o[r] = __ldg(&kOffsetTable.w[nb_index<NB>()][order_index<GSV>()][r][lane]);
     }
     // table byte offset of the entry step q selects: (pattern << 8) | bank*4
     __device__ __forceinline__ uint32_t addr(uint32_t w, int q) const {
@@ -262,6 +280,34 @@ __device__ __forceinline__ void lookup_unit(const uint4 (&w)[Geom<MU, BT>::kVecs
     for (int b = 0; b < BT; ++b)
 #pragma unroll
         for (int i = 0; i < NB; ++i) acc[b][i] += sum_f32x2(pair[b][i]);
+}
+
+// Salient branch with row scales per group of GSV sub-vectors (grouped visit
+// order): after the GSV steps of slot a the lane has the whole contribution of
+// one (base, group) to its row and multiplies it by that group's row scale,
+// staged in shared memory in slot order.  One batch row (BT == 1).
+template <int MU, int NB, int GSV, int HALF>
+__device__ __forceinline__ void lookup_unit_grouped(const uint4 (&w)[kSlabsPerWarp][Geom<MU, 1>::kVecs],
+                                                    const Offsets<MU>& off, uint32_t tbase, uint32_t scale_row_off,
+                                                    float (&tot)[kSlabsPerWarp][1]) {
+    constexpr int kStepsPerWord = 32 / MU;
+    constexpr int KG = 32 / GSV;
+#pragma unroll
+    for (int a = 0; a < KG; ++a) {
+#pragma unroll
+        for (int rs = 0; rs < kSlabsPerWarp; ++rs) {
+            float g = 0.f;
+#pragma unroll
+            for (int e = 0; e < GSV; ++e) {
+                const int q = a * GSV + e;
+                const int wi = q / kStepsPerWord;
+                g += lds_f32<HALF * 128>(tbase + off.addr(word_of(w[rs][wi / 4], wi % 4), q));
+            }
+            const float sc = __half2float(
+                smem_at<const __half>(scale_row_off + (uint32_t)(a * kRowsPerCta + rs * kLanes) * 2u));
+            tot[rs][0] = fmaf(sc, g, tot[rs][0]);
+        }
+    }
 }
 
 // The activation-product slot a thread owns: bank c = s / mu, bit t = s % mu.
@@ -378,17 +424,40 @@ struct WeightRegs {
     uint4 w[2][kSlabsPerWarp][Geom<MU, BT>::kVecs];
 };
 
+// Row scales of the grouped salient branch for unit u (a salient unit),
+// staged for parity `par` in slot order: entry [a][row] is the scale of the
+// (base, group) lane L = row % 32 completes at slot a.
+template <int MU, int NB1, int GS1>
+__device__ __forceinline__ void stage_group_scales(const KernelArgs& a, int u, int rg, int tid, int par) {
+    if constexpr (GS1 > 0) {
+        constexpr int P = 32 / NB1, NG = P / GS1, KG = 32 / GS1;
+        const int ul = u - a.br[0].units;
+        const __half* r = a.br[1].r;
+        const int ng = a.br[1].ngroups;
+#pragma unroll 8
+        for (int e = tid; e < KG * kRowsPerCta; e += kThreads) {
+            const int slot = e / kRowsPerCta, lrow = e % kRowsPerCta;
+            const int kg = visit_group(lrow % kLanes, slot, GS1);
+            const int k = kg / NG, gg = ul * NG + kg % NG;
+            const int row = rg * kRowsPerCta + lrow;
+            const __half v = (row < a.M && gg < ng) ? r[((int64_t)k * ng + gg) * a.M + row] : __float2half(0.f);
+            smem_at<__half>(Geom<MU, 1>::kScaleOff + (uint32_t)((par * KG + slot) * kRowsPerCta + lrow) * 2u) = v;
+        }
+    }
+}
+
 // One unit of branch BR: build its tables, form the next unit's products and
 // request the inputs two units ahead, then every slab's lookups, refilling
 // each slab's registers with the unit two ahead as soon as they are consumed.
-template <int MU, int BR, int NB, int HALF, int BT, int NB0, int NB1>
-__device__ __forceinline__ void unit_step(const KernelArgs& a, int u, int u_end, int ul, int b0, int slab0,
+template <int MU, int BR, int NB, int HALF, int BT, int NB0, int NB1, int GS1>
+__device__ __forceinline__ void unit_step(const KernelArgs& a, int u, int u_end, int ul, int b0, int rg, int slab0,
                                           int warp, int lane, int tid, uint32_t sbase, const Offsets<MU>& off,
                                           ProductPipe<BT>& pp, WeightRegs<MU, BT>& wb,
                                           float (&acc)[kSlabsPerWarp][BT][NB],
                                           float (&tot)[kSlabsPerWarp][BT]) {
     const BranchArgs& br = a.br[BR];
     constexpr int P = 32 / NB;
+    constexpr bool kGrouped = BR == 1 && GS1 > 0;
     build_unit<MU, HALF, BT>(sbase, warp, lane);
     if (tid < Geom<MU, BT>::kSlots && u + 1 < u_end) {
         store_products<MU, BT>(sbase, HALF ^ 1, tid, pp.c1, pp.x1);
@@ -401,7 +470,7 @@ __device__ __forceinline__ void unit_step(const KernelArgs& a, int u, int u_end,
         }
     }
     float rsc[kSlabsPerWarp][NB];
-    if (br.rgroup > 0) {
+    if (!kGrouped && br.rgroup > 0) {
         const int g = (int)(((int64_t)ul * P * MU) / br.rgroup);
 #pragma unroll
         for (int rs = 0; rs < kSlabsPerWarp; ++rs) {
@@ -414,15 +483,34 @@ __device__ __forceinline__ void unit_step(const KernelArgs& a, int u, int u_end,
         }
     }
     __syncthreads();
-#pragma unroll
-    for (int rs = 0; rs < kSlabsPerWarp; ++rs) {
-        uint4 cur[Geom<MU, BT>::kVecs];
-#pragma unroll
-        for (int h = 0; h < Geom<MU, BT>::kVecs; ++h) cur[h] = wb.w[HALF][rs][h];
-        if (u + 2 < u_end) load_unit_slab<MU, BT>(a, u + 2, slab0 + rs, lane, wb.w[HALF][rs]);
-        lookup_unit<MU, NB, HALF, BT>(cur, off, sbase, acc[rs]);
+    if constexpr (GS1 > 0) {
+        // every warp is past the lookups of unit u-1, whose scale buffer this
+        // reuses; the next barrier publishes it for unit u+1
+        if (u + 1 < u_end && u + 1 >= a.br[0].units) stage_group_scales<MU, NB1, GS1>(a, u + 1, rg, tid, HALF ^ 1);
     }
-    if (br.rgroup > 0) {
+    if constexpr (kGrouped) {
+        static_assert(BT == 1, "grouped salient scales are built for one batch row per CTA");
+        uint4 cur[kSlabsPerWarp][Geom<MU, BT>::kVecs];
+#pragma unroll
+        for (int rs = 0; rs < kSlabsPerWarp; ++rs) {
+#pragma unroll
+            for (int h = 0; h < Geom<MU, BT>::kVecs; ++h) cur[rs][h] = wb.w[HALF][rs][h];
+            if (u + 2 < u_end) load_unit_slab<MU, BT>(a, u + 2, slab0 + rs, lane, wb.w[HALF][rs]);
+        }
+        const uint32_t scale_row_off = Geom<MU, 1>::kScaleOff +
+            (uint32_t)((HALF * (32 / GS1)) * kRowsPerCta + (slab0 % kSlabsPerCta) * kLanes + lane) * 2u;
+        lookup_unit_grouped<MU, NB, GS1, HALF>(cur, off, sbase, scale_row_off, tot);
+    } else {
+#pragma unroll
+        for (int rs = 0; rs < kSlabsPerWarp; ++rs) {
+            uint4 cur[Geom<MU, BT>::kVecs];
+#pragma unroll
+            for (int h = 0; h < Geom<MU, BT>::kVecs; ++h) cur[h] = wb.w[HALF][rs][h];
+            if (u + 2 < u_end) load_unit_slab<MU, BT>(a, u + 2, slab0 + rs, lane, wb.w[HALF][rs]);
+            lookup_unit<MU, NB, HALF, BT>(cur, off, sbase, acc[rs]);
+        }
+    }
+    if (!kGrouped && br.rgroup > 0) {
         // block-wise row scales: the unit lies in one column block
 #pragma unroll
         for (int rs = 0; rs < kSlabsPerWarp; ++rs)
@@ -436,23 +524,23 @@ __device__ __forceinline__ void unit_step(const KernelArgs& a, int u, int u_end,
     }
 }
 
-template <int MU, int BR, int NB, int BT, int NB0, int NB1>
-__device__ __forceinline__ void run_branch(const KernelArgs& a, int u_lo, int u_hi, int u_end, int& v, int b0,
+template <int MU, int BR, int NB, int BT, int NB0, int NB1, int GS1>
+__device__ __forceinline__ void run_branch(const KernelArgs& a, int u_lo, int u_hi, int u_end, int& v, int b0, int rg,
                                            int slab0, int warp, int lane, int tid, uint32_t sbase,
                                            ProductPipe<BT>& pp, WeightRegs<MU, BT>& wb,
                                            float (&acc)[kSlabsPerWarp][BT][NB],
                                            float (&tot)[kSlabsPerWarp][BT]) {
     if (u_lo >= u_hi) return;
     Offsets<MU> off;
-    off.template load<NB>(lane);
+    off.template load<NB, BR == 1 ? GS1 : 0>(lane);
     const int ubase = BR ? a.br[0].units : 0;
     for (int u = u_lo; u < u_hi; ++u, ++v) {
         if (v & 1)
-            unit_step<MU, BR, NB, 1, BT, NB0, NB1>(a, u, u_end, u - ubase, b0, slab0, warp, lane, tid, sbase, off, pp,
-                                                   wb, acc, tot);
+            unit_step<MU, BR, NB, 1, BT, NB0, NB1, GS1>(a, u, u_end, u - ubase, b0, rg, slab0, warp, lane, tid, sbase,
+                                                        off, pp, wb, acc, tot);
         else
-            unit_step<MU, BR, NB, 0, BT, NB0, NB1>(a, u, u_end, u - ubase, b0, slab0, warp, lane, tid, sbase, off, pp,
-                                                   wb, acc, tot);
+            unit_step<MU, BR, NB, 0, BT, NB0, NB1, GS1>(a, u, u_end, u - ubase, b0, rg, slab0, warp, lane, tid, sbase,
+                                                        off, pp, wb, acc, tot);
     }
 }
 
@@ -489,7 +577,7 @@ __device__ __forceinline__ void store_y(const KernelArgs& a, int b, int i, float
 template <int BT>
 constexpr int min_blocks() { return BT == 1 ? 2 : 1; }
 
-template <int MU, int NB0, int NB1, int BT>
+template <int MU, int NB0, int NB1, int BT, int GS1>
 __global__ void __launch_bounds__(kThreads, min_blocks<BT>()) fluxbin_lut_kernel(const KernelArgs a) {
     using G = Geom<MU, BT>;
     constexpr int NB1E = NB1 > 0 ? NB1 : 1;
@@ -540,6 +628,11 @@ __global__ void __launch_bounds__(kThreads, min_blocks<BT>()) fluxbin_lut_kernel
         slot_x<BT>(a, b0, st0.col, x0);
         slot_x<BT>(a, b0, st1.col, pp.x1);
         if (u_begin < u_end) store_products<MU, BT>(sbase, 0, tid, st0.c, x0);
+    }
+    if constexpr (GS1 > 0) {
+        if (u_begin < u_end && u_begin >= U0) stage_group_scales<MU, NB1, GS1>(a, u_begin, rg, tid, 0);
+    }
+    if (slot_owner) {
         pp.c1 = st1.c;
         pp.c2 = st2.c;
         pp.col2 = st2.col;
@@ -561,11 +654,11 @@ __global__ void __launch_bounds__(kThreads, min_blocks<BT>()) fluxbin_lut_kernel
         }
 
     int v = 0;
-    run_branch<MU, 0, NB0, BT, NB0, NB1>(a, u_begin, min(u_end, U0), u_end, v, b0, slab0, warp, lane, tid, sbase,
-                                         pp, wb, acc0, tot);
+    run_branch<MU, 0, NB0, BT, NB0, NB1, GS1>(a, u_begin, min(u_end, U0), u_end, v, b0, rg, slab0, warp, lane, tid,
+                                              sbase, pp, wb, acc0, tot);
     if constexpr (NB1 > 0)
-        run_branch<MU, 1, NB1, BT, NB0, NB1>(a, max(u_begin, U0), u_end, u_end, v, b0, slab0, warp, lane, tid, sbase,
-                                             pp, wb, acc1, tot);
+        run_branch<MU, 1, NB1, BT, NB0, NB1, GS1>(a, max(u_begin, U0), u_end, u_end, v, b0, rg, slab0, warp, lane, tid,
+                                                  sbase, pp, wb, acc1, tot);
 
     // Row scales (per-row case; the block-wise case was applied per unit).
 #pragma unroll

@@ -38,20 +38,52 @@ FB_HD int64_t branch_words(int64_t M, int64_t ncols, int nb, int mu) {
     return row_slabs(M) * branch_units(ncols, nb, mu) * chunk_words(mu);
 }
 
-// Step at which lane L visits (base k, sub-vector j of the unit).
-FB_HD int visit_step(int L, int k, int j, int nb) {
+// Sub-vectors per row-scale group inside a unit (gsv).  A branch whose scales
+// change every gsv < P sub-vectors uses the grouped visit order below; every
+// other branch uses the plain diagonal order (gsv == P).
+FB_HD int group_subvecs(int nb, int mu, int scale_group) {
     const int P = subvecs_per_unit(nb);
-    const int a = ((k - L / P) % nb + nb) % nb;
-    const int d = ((j - L) % P + P) % P;
-    return a * P + d;
+    return (scale_group > 0 && scale_group < P * mu) ? scale_group / mu : P;
 }
-// Bank (table slot) that lane L reads at step q: base k = (q/P + L/P) mod nb,
-// sub-vector j = (L + q) mod P, slot k*P + j.
-FB_HD int visit_bank(int L, int q, int nb) {
+
+// Step at which lane L visits (base k, sub-vector j of the unit).
+//   diagonal (gsv == P): k = (q/P + L/P) mod nb, j = (L + q) mod P
+//   grouped  (gsv <  P): lane L = gsv*m + s, step q = gsv*a + e;
+//                        kg = (a + m) mod (32/gsv), k = kg / (P/gsv),
+//                        j = gsv*(kg mod (P/gsv)) + (e xor s)
+FB_HD int visit_step(int L, int k, int j, int nb, int gsv) {
     const int P = subvecs_per_unit(nb);
-    const int k = (q / P + L / P) % nb;
-    const int j = (L + q) % P;
-    return k * P + j;
+    if (gsv >= P) {
+        const int a = ((k - L / P) % nb + nb) % nb;
+        const int d = ((j - L) % P + P) % P;
+        return a * P + d;
+    }
+    const int KG = kLanes / gsv, NG = P / gsv;
+    const int m = L / gsv, sg = L % gsv;
+    const int e = (j % gsv) ^ sg;
+    const int kg = k * NG + j / gsv;
+    const int a = ((kg - m) % KG + KG) % KG;
+    return a * gsv + e;
+}
+// Bank (table slot k*P + j) that lane L reads at step q.
+FB_HD int visit_bank(int L, int q, int nb, int gsv) {
+    const int P = subvecs_per_unit(nb);
+    if (gsv >= P) {
+        const int k = (q / P + L / P) % nb;
+        const int j = (L + q) % P;
+        return k * P + j;
+    }
+    const int KG = kLanes / gsv, NG = P / gsv;
+    const int m = L / gsv, sg = L % gsv;
+    const int a = q / gsv, e = q % gsv;
+    const int kg = (a + m) % KG;
+    return (kg / NG) * P + gsv * (kg % NG) + (e ^ sg);
+}
+// Group (base k, scale group g of the unit) whose sum lane L completes at
+// slot a = q / gsv of the grouped order: returned as kg = k*(P/gsv) + g.
+FB_HD int visit_group(int L, int a, int gsv) {
+    const int KG = kLanes / gsv;
+    return (a + L / gsv) % KG;
 }
 
 }  // namespace fluxbin

@@ -13,8 +13,9 @@ using namespace fluxbin;
 
 namespace {
 
-// Packs one branch: signs [nb][M][ncols] (+-1) -> words (device layout).
-int pack_branch(const int8_t* signs, int64_t M, int64_t ncols, int nb, int mu, uint32_t* words) {
+// Packs one branch: signs [nb][M][ncols] (+-1) -> words (device layout);
+// gsv selects the visit order (see fluxbin_layout.h).
+int pack_branch(const int8_t* signs, int64_t M, int64_t ncols, int nb, int mu, int gsv, uint32_t* words) {
     const int P = subvecs_per_unit(nb);
     const int64_t U = branch_units(ncols, nb, mu);
     const int64_t total = branch_words(M, ncols, nb, mu);
@@ -36,7 +37,7 @@ int pack_branch(const int8_t* signs, int64_t M, int64_t ncols, int nb, int mu, u
                 if (!pat) continue;
                 const int64_t u = jg / P;
                 const int j = (int)(jg % P);
-                const int q = visit_step(L, k, j, nb);
+                const int q = visit_step(L, k, j, nb, gsv);
                 const int pos = q * mu;
                 const int64_t w = (s * U + u) * chunk_words(mu) + ((int64_t)(pos / 128) * kLanes + L) * 4 + (pos / 32) % 4;
                 words[w] |= pat << (pos % 32);
@@ -92,11 +93,12 @@ int fluxbin_pack(const fluxbin_layer_desc* desc, const int8_t* signs, const int8
         }
     }
     if (nw > 0) {
-        const int r = pack_branch(signs, d.M, d.N, d.Kb, d.mu, words_out);
+        const int r = pack_branch(signs, d.M, d.N, d.Kb, d.mu, subvecs_per_unit(d.Kb), words_out);
         if (r != FLUXBIN_OK) return r;
     }
     if (has_salient(d) && branch_words(d.M, d.n_sal, d.Ks, d.mu) > 0) {
-        const int r = pack_branch(sal_signs, d.M, d.n_sal, d.Ks, d.mu, swords_out);
+        const int r = pack_branch(sal_signs, d.M, d.n_sal, d.Ks, d.mu, group_subvecs(d.Ks, d.mu, d.sal_scale_group),
+                                  swords_out);
         if (r != FLUXBIN_OK) return r;
     }
     return FLUXBIN_OK;

@@ -14,6 +14,9 @@ Definition (one branch: nb bases, ncols columns, M rows, sub-vector length mu):
     u, j  = jg // P, jg % P
     a     = (k - L // P) mod nb
     q     = a*P + ((j - L) mod P)           visit step of that sub-vector for lane L
+  (grouped order, for a branch whose row scales change every gsv < P
+   sub-vectors: KG = 32/gsv, NG = P/gsv, m, g = L // gsv, L % gsv,
+    kg = k*NG + j // gsv, a = (kg - m) mod KG, q = a*gsv + ((j mod gsv) xor g))
     pos   = q*mu + t
     word  = (s*U + u)*(32*mu) + ((pos // 128)*32 + L)*4 + (pos // 32) % 4
     bit   = pos % 32
@@ -35,7 +38,7 @@ def branch_words(M: int, ncols: int, nb: int, mu: int) -> int:
     return Ms * U * 32 * mu
 
 
-def _positions(M: int, ncols: int, nb: int, mu: int):
+def _positions(M: int, ncols: int, nb: int, mu: int, gsv: int = 0):
     P, U, Ms = branch_geometry(M, ncols, nb, mu)
     k = np.arange(nb, dtype=np.int64)[:, None, None]
     i = np.arange(M, dtype=np.int64)[None, :, None]
@@ -43,8 +46,15 @@ def _positions(M: int, ncols: int, nb: int, mu: int):
     s, L = i // 32, i % 32
     jg, t = n // mu, n % mu
     u, j = jg // P, jg % P
-    a = np.mod(k - L // P, nb)
-    q = a * P + np.mod(j - L, P)
+    if gsv and gsv < P:
+        KG, NG = 32 // gsv, P // gsv
+        m, sg = L // gsv, L % gsv
+        kg = k * NG + j // gsv
+        a = np.mod(kg - m, KG)
+        q = a * gsv + np.bitwise_xor(j % gsv, sg)
+    else:
+        a = np.mod(k - L // P, nb)
+        q = a * P + np.mod(j - L, P)
     pos = q * mu + t
     word = (s * U + u) * (32 * mu) + ((pos // 128) * 32 + L) * 4 + (pos // 32) % 4
     bit = pos % 32
@@ -52,23 +62,24 @@ def _positions(M: int, ncols: int, nb: int, mu: int):
     return word, bit
 
 
-def pack_branch(signs: np.ndarray, mu: int) -> np.ndarray:
-    """signs int8 [nb][M][ncols] (+-1) -> uint32 words of the device layout."""
+def pack_branch(signs: np.ndarray, mu: int, gsv: int = 0) -> np.ndarray:
+    """signs int8 [nb][M][ncols] (+-1) -> uint32 words of the device layout
+    (gsv: sub-vectors per row-scale group for the grouped visit order)."""
     nb, M, ncols = signs.shape
     total = branch_words(M, ncols, nb, mu)
     out = np.zeros(total, dtype=np.uint64)
     if total == 0:
         return out.astype(np.uint32)
-    word, bit = _positions(M, ncols, nb, mu)
+    word, bit = _positions(M, ncols, nb, mu, gsv)
     plus = signs > 0
     # every (word, bit) pair is distinct, so adding the set bits is an OR
     np.add.at(out, word[plus], np.left_shift(np.uint64(1), bit[plus].astype(np.uint64)))
     return out.astype(np.uint32)
 
 
-def unpack_branch(words: np.ndarray, M: int, ncols: int, nb: int, mu: int) -> np.ndarray:
+def unpack_branch(words: np.ndarray, M: int, ncols: int, nb: int, mu: int, gsv: int = 0) -> np.ndarray:
     """Inverse of pack_branch: uint32 words -> int8 signs [nb][M][ncols]."""
-    word, bit = _positions(M, ncols, nb, mu)
+    word, bit = _positions(M, ncols, nb, mu, gsv)
     w = np.asarray(words, dtype=np.uint32)
     bits = (w[word] >> bit.astype(np.uint32)) & 1
     return (bits.astype(np.int8) * 2 - 1).astype(np.int8)

@@ -64,6 +64,24 @@ def test_pack_bit_exact_against_naive_packer(M, N, Kb, Ks, n_sal, mu):
     del rng
 
 
+@pytest.mark.parametrize("M,N,Kb,Ks,n_sal,mu,Gs,gsv", [
+    (70, 512, 2, 2, 64, 8, 16, 2), (33, 300, 1, 1, 100, 8, 8, 1), (64, 1024, 2, 4, 96, 8, 32, 4),
+    (40, 256, 2, 2, 64, 4, 8, 2), (50, 512, 4, 1, 60, 4, 16, 4), (32, 4096, 2, 2, 512, 8, 16, 2)])
+def test_pack_grouped_salient_bit_exact(M, N, Kb, Ks, n_sal, mu, Gs, gsv):
+    """Salient row scales finer than a unit use the grouped visit order."""
+    spec = LayerSpec("g", M, N, Kb, Ks, n_sal, mu, sal_scale_group=Gs)
+    d = make_layer(spec, [M, N, Gs])
+    desc = LayerDesc.of(spec)
+    words, swords = fluxbin.fluxbin_pack(desc, d.signs, d.sal_signs, d.sal_idx)
+    assert np.array_equal(words, layout.pack_branch(d.signs, mu))
+    assert np.array_equal(swords, layout.pack_branch(d.sal_signs, mu, gsv))
+    assert np.array_equal(layout.unpack_branch(swords, M, n_sal, Ks, mu, gsv), d.sal_signs)
+    # a different permutation of the same bits, except for one base with one
+    # sub-vector per group, where both orders are the plain diagonal
+    same = np.array_equal(swords, layout.pack_branch(d.sal_signs, mu))
+    assert same == (Ks == 1 and gsv == 1)
+
+
 def test_pack_rejects_bad_inputs():
     spec = LayerSpec("p", 8, 64, 1, 1, 4, 8)
     d = make_layer(spec, [1])
@@ -81,7 +99,8 @@ def test_pack_rejects_bad_inputs():
 
 @pytest.mark.parametrize("field,value,status", [
     ("mu", 5, -4), ("mu", 16, -4), ("Kb", 3, -4), ("Kb", 0, -4), ("Ks", 3, -4), ("M", -1, -2),
-    ("n_sal", 70, -2), ("row_scale_group", 100, -4), ("row_scale_group", -2, -2)])
+    ("n_sal", 70, -2), ("row_scale_group", 100, -4), ("row_scale_group", -2, -2),
+    ("sal_scale_group", 12, -4), ("sal_scale_group", 24, -4), ("sal_scale_group", 64, -4)])
 def test_desc_validation(field, value, status):
     desc = LayerDesc(32, 64, 2, 1, 4, 8, 0, 0)
     setattr(desc, field, value)

@@ -89,6 +89,13 @@ CASES = [
     (spec(64, 2048, 2, 0, 0, 8, G=128), 1),  # block-wise row scales
     (spec(1100, 1024, 2, 1, 64, 4, G=128), 3),
     (spec(1100, 1024, 1, 0, 0, 8, G=256), 2),
+    (spec(2100, 1024, 2, 2, 128, 8, G=128, sal_scale_group=16, sal_per_group=16), 1),  # 2.75-bit layout
+    (spec(1100, 777, 2, 2, 120, 8, sal_scale_group=16), 3),
+    (spec(1100, 777, 1, 1, 120, 8, sal_scale_group=8), 2),
+    (spec(1100, 777, 2, 4, 120, 8, sal_scale_group=32), 1),
+    (spec(900, 600, 2, 2, 100, 4, sal_scale_group=8), 2),
+    (spec(900, 600, 1, 1, 100, 4, sal_scale_group=4), 1),
+    (spec(900, 600, 4, 2, 100, 4, sal_scale_group=16), 1),
     (spec(256, 65536, 2, 1, 300, 8), 1),     # split wider than a cluster: workspace path
     (spec(100, 30000, 1, 2, 500, 4), 3),
     (spec(4096, 4096, 2, 1, 205, 8), 2),
@@ -107,7 +114,9 @@ def test_parity_random(sp, B):
 @pytest.mark.parametrize("mu", [4, 8])
 def test_exact_arithmetic_is_bit_exact(mu):
     for i, (sp, B) in enumerate([(spec(2100, 777, 2, 1, 40, mu), 3), (spec(1030, 1500, 1, 2, 100, mu), 1),
-                                 (spec(300, 512, 2, 0, 0, mu, G=128), 2)]):
+                                 (spec(300, 512, 2, 0, 0, mu, G=128), 2),
+                                 (spec(700, 1024, 2, 2, 128, mu, G=128, sal_scale_group=2 * mu,
+                                       sal_per_group=16), 2)]):
         layer = synth.make_exact_layer(sp, [80, i, mu])
         x = synth.make_exact_x(sp, B, [81, i, mu])
         ref = oracle.linear(layer, x)
