@@ -41,7 +41,7 @@ size_t table_smem_bytes(int mu, int bt) {
 // per slot (32/gs1 of them) and row of the CTA.
 size_t scale_smem_bytes(int gs1) { return gs1 > 0 ? 2u * (32u / (size_t)gs1) * kRowsPerCta * 2u : 0u; }
 // Cluster reduction buffer: one fp32 partial per row of the CTA and batch row.
-size_t red_smem_bytes(int bt) { return (size_t)bt * kRowsPerCta * sizeof(float); }
+size_t red_smem_bytes(int bt) { return (size_t)bt * kRedRows * sizeof(float); }
 
 struct DeviceInfo {
     int sm_count = 0;

@@ -42,7 +42,8 @@
 //           parity h at b*2^mu*256 + e*256 + h*128 + bank*4 (consecutive units
 //           alternate halves: double buffering with one barrier per unit)
 //   vbuf    2 * BT * 32*mu floats: [parity][b][bank][t] activation products
-//   red     BT * 512 floats: partial sums for the cluster reduction
+//   red     BT * 528 floats: [b][source rank][row of this CTA's slice], the
+//           split-K partials the cluster's CTAs push to the slice owner
 //   scales  (grouped salient branch only) 2 * (32/gsv) * 512 fp16: the row
 //           scale each lane applies after each group, [parity][slot][row]
 #pragma once
@@ -97,7 +98,7 @@ struct Geom {
     static constexpr int kVbufOff = kTableBytes;
     static constexpr int kVbufBytes = 2 * BT * kSlots * 4;
     static constexpr int kRedOff = kVbufOff + kVbufBytes;
-    static constexpr int kRedBytes = BT * kRowsPerCta * 4;
+    static constexpr int kRedBytes = BT * kRedRows * 4;
     static constexpr int kScaleOff = kRedOff + kRedBytes;  // grouped salient branch: staged scales
 };
 
@@ -202,13 +203,11 @@ __device__ __forceinline__ uint32_t cluster_rank() {
     return r;
 }
 
-// Load a float from the same shared-memory offset in CTA `rank` of the cluster.
-__device__ __forceinline__ float ld_dsmem_f32(uint32_t local_smem_addr, uint32_t rank) {
+// Store a float at a shared-memory offset in CTA `rank` of the cluster.
+__device__ __forceinline__ void st_dsmem_f32(uint32_t local_smem_addr, uint32_t rank, float v) {
     uint32_t ra;
     asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(local_smem_addr), "r"(rank));
-    float v;
-    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(ra) : "memory");
-    return v;
+    asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(ra), "f"(v) : "memory");
 }
 
 template <int MU>
@@ -687,32 +686,34 @@ __global__ void __launch_bounds__(kThreads, min_blocks<BT>()) fluxbin_lut_kernel
     }
 
     if (a.cluster) {
-        // Split-K reduction inside the cluster: every CTA parks its partials in
-        // its own shared memory; CTA r then sums slice r of the rows over all
-        // CTAs in rank order and writes y.
+        // Split-K reduction inside the cluster: CTA r owns rows [r*chunk,
+        // (r+1)*chunk) of the row group.  Every CTA pushes each partial to the
+        // owner's shared memory, slot [b][own rank][row - r*chunk]; one cluster
+        // barrier publishes the stores; each owner then sums its slots in rank
+        // order from local memory (deterministic) and writes y.
+        const int C = a.n_ks;
+        const int rank = (int)cluster_rank();
+        const int chunk = (kRowsPerCta + C - 1) / C;
         const uint32_t red = sbase + G::kRedOff;
 #pragma unroll
         for (int rs = 0; rs < kSlabsPerWarp; ++rs) {
             const int lr = (warp * kSlabsPerWarp + rs) * kLanes + lane;
+            const int owner = lr / chunk, j = lr % chunk;
 #pragma unroll
-            for (int b = 0; b < BT; ++b) sts_f32(red + (uint32_t)(b * kRowsPerCta + lr) * 4u, tot[rs][b]);
+            for (int b = 0; b < BT; ++b)
+                st_dsmem_f32(red + (uint32_t)((b * C + rank) * chunk + j) * 4u, (uint32_t)owner, tot[rs][b]);
         }
         cluster_sync_all();
-        const int C = a.n_ks;
-        const int rank = (int)cluster_rank();
-        const int chunk = (kRowsPerCta + C - 1) / C;
         for (int e = tid; e < BT * chunk; e += kThreads) {
-            const int b = e / chunk, lr = rank * chunk + e % chunk;
-            if (lr >= kRowsPerCta) continue;
+            const int b = e / chunk, j = e % chunk, lr = rank * chunk + j;
             const int i = row0 + lr;
-            if (i >= a.M || b0 + b >= a.B) continue;
-            const uint32_t off = red + (uint32_t)(b * kRowsPerCta + lr) * 4u;
+            if (lr >= kRowsPerCta || i >= a.M || b0 + b >= a.B) continue;
+            const float* slot = &smem_at<const float>(G::kRedOff + (uint32_t)(b * C * chunk + j) * 4u);
             float s = 0.f;
-            for (int c = 0; c < C; ++c) s += ld_dsmem_f32(off, (uint32_t)c);
+#pragma unroll 16
+            for (int c = 0; c < C; ++c) s += slot[c * chunk];
             store_y(a, b0 + b, i, s);
         }
-        // keep every CTA's shared memory alive until all reads are done
-        cluster_sync_all();
         return;
     }
 

@@ -20,6 +20,8 @@ constexpr int kSlabsPerWarp = 2;    // row slabs a warp keeps accumulators for
 constexpr int kSlabsPerCta = kWarps * kSlabsPerWarp;
 constexpr int kRowsPerCta = kSlabsPerCta * kLanes;  // 512
 constexpr int kMaxCluster = 16;     // CTAs that reduce their split-K partials through DSMEM
+// partial sums a CTA receives in a cluster reduction: C slices of ceil(512/C) rows
+constexpr int kRedRows = kRowsPerCta + kMaxCluster;
 constexpr int kMaxBatch = 16;
 
 // Sub-vectors of one base inside a unit.
