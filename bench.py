@@ -508,6 +508,116 @@ def run_sweep(device, l2, args):
     return out
 
 
+# ----------------------------------------------------------------------------
+# The LLaMA-2-7B-shaped decoder stack (32 x q,k,v,o,gate,up,down), 2.75 bits
+# ----------------------------------------------------------------------------
+
+def _stack_job(job):
+    """Worker: draw and pack one linear of the stack (host only)."""
+    l, li = job
+    from lut_binary_basis_b200 import fluxbin, synth
+    sp = synth.layers_7b_stack_linears()[li]
+    host = synth.make_layer(sp, synth.layer_key(4, l, li))
+    packed = fluxbin.pack_host(host)
+    x = synth.make_x(sp, 1, synth.x_key(4, l, li, 1))
+    return l, li, packed, x
+
+
+def build_stack(device, n_layers, workers):
+    """Every linear of the stack resident on the device, with its own seeded
+    fp16 N(0,1) input and fp16 output (the linears are chained in order but do
+    not feed one another: without the normalisation and attention between
+    them the outputs would overflow fp16)."""
+    import multiprocessing as mp
+    import torch
+    from lut_binary_basis_b200 import fluxbin, synth
+    specs = synth.layers_7b_stack_linears()
+    jobs = [(l, li) for l in range(n_layers) for li in range(len(specs))]
+    out = []
+    with mp.get_context("spawn").Pool(workers) as pool:
+        for l, li, packed, x in pool.imap(_stack_job, jobs, chunksize=1):
+            sp = specs[li]
+            out.append((sp, fluxbin.DeviceLayer.from_packed(packed, device), torch.from_numpy(x).to(device),
+                        torch.empty((1, sp.M), dtype=torch.float16, device=device)))
+    return out
+
+
+def stack_bits_per_weight(specs) -> float:
+    """Packed bits + fp16 scales + int32 column map per weight of the stack's linears."""
+    bits = w = 0
+    for sp in specs:
+        bits += 8 * (algorithmic_bytes(sp, 1) - 2 * sp.N - 2 * sp.M)
+        w += sp.M * sp.N
+    return bits / w
+
+
+def run_stack(args):
+    """One decode step (batch 1) through all 224 linears, chained in order
+    under one CUDA graph; a step's inputs are resident and the weights (2.2 GB)
+    are far larger than L2."""
+    import torch
+    import __graft_entry__
+    from lut_binary_basis_b200 import fluxbin, synth
+    __graft_entry__.build()
+    n_layers = args.stack_layers
+    workers = max(1, min(8, (os.cpu_count() or 2) - 1))
+    t0 = time.time()
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    layers = build_stack(device, n_layers, workers)
+    setup_s = time.time() - t0
+    ws = fluxbin.new_workspace(max(sp.M for sp, *_ in layers), 1, device)
+    flags = fluxbin.FLAG_EARLY_WEIGHTS
+    stream = torch.cuda.Stream(device)
+
+    def step():
+        for sp, dl, x, y in layers:
+            dl.linear(x, y, flags, ws, stream)
+
+    with torch.cuda.stream(stream):
+        step()
+    stream.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        step()
+    for _ in range(args.warmup):
+        g.replay()
+    torch.cuda.synchronize(device)
+    props = torch.cuda.get_device_properties(device)
+    sampler = ClockSampler(gpu_id_for_smi(props)) if not args.no_clocks else None
+    if sampler:
+        sampler.start()
+        time.sleep(0.2)
+        sampler.mark(True)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    with torch.cuda.stream(stream):
+        for _ in range(args.steps):
+            g.replay()
+    e1.record(stream)
+    torch.cuda.synchronize(device)
+    if sampler:
+        sampler.mark(False)
+        sampler.stop()
+    secs = e0.elapsed_time(e1) / 1e3 / args.steps
+    total = sum(algorithmic_bytes(sp, 1) for sp, *_ in layers)
+    peak, peak_kind = measured_peaks()
+    gbs = total / secs / 1e9
+    specs = synth.layers_7b_stack_linears()
+    return {"metric": "LLaMA-2-7B-shaped decoder stack, linears only: decode step time (batch 1)",
+            "value": secs * 1e6, "unit": "us/token", "higher_is_better": False, "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup, "tokens_per_s": 1.0 / secs,
+            "dtype": "f32", "data": "synthetic (seeded)",
+            "config": {"workload": "llama7b_stack_32x7_275bit_b1", "layers": n_layers,
+                       "linears": len(layers), "bits_per_weight": stack_bits_per_weight(specs),
+                       "graph": "one CUDA graph, linears chained in order with programmatic dependent launch",
+                       "l2_policy": f"weights {total / 2**30:.2f} GiB per step > L2"},
+            "achieved_gbs": gbs, "roofline": {"bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s",
+                                              "frac": gbs / peak, "peak_source": peak_kind},
+            "gpu_launches": len(layers) * args.steps, "setup_s": setup_s,
+            "clocks": sampler.summary() if sampler else None}
+
+
 def run_reference(args, rank, world):
     """The oracle (CPU, all host cores) on a bounded sample of the same layer."""
     if rank != 0:
@@ -547,11 +657,17 @@ def main(argv=None):
     ap.add_argument("--layer", default=None,
                     help="time one named layer of the workloads instead (e.g. llama7b_gate_up_11008x4096)")
     ap.add_argument("--batch", type=int, default=1)
+    ap.add_argument("--stack", action="store_true",
+                    help="time the 32-layer LLaMA-2-7B-shaped stack of 2.75-bit linears instead")
+    ap.add_argument("--stack-layers", type=int, default=32)
     args = ap.parse_args(argv)
     args.warmup = max(3, args.warmup)
     rank, local_rank, world = dist_env()
     if args.layer:
         print(json.dumps(run_one_layer(args)), flush=True)
+        return
+    if args.stack:
+        print(json.dumps(run_stack(args)), flush=True)
         return
     if args.impl == "reference":
         res = run_reference(args, rank, world)

@@ -45,7 +45,7 @@
 //   red     BT * 528 floats: [b][source rank][row of this CTA's slice], the
 //           split-K partials the cluster's CTAs push to the slice owner
 //   scales  (grouped salient branch only) 2 * (32/gsv) * 512 fp16: the row
-//           scale each lane applies after each group, [parity][slot][row]
+//           scales of each (base, group) of the unit, [parity][group][row]
 #pragma once
 
 #include <cuda_fp16.h>
@@ -189,6 +189,12 @@ __device__ __forceinline__ float sum_f32x2(uint64_t x) {
     return lo + hi;
 }
 
+__device__ __forceinline__ void cp_async16(uint32_t smem_addr, const void* gptr) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_addr), "l"(gptr) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+
 __device__ __forceinline__ void red_add_f32(float* p, float v) {
     asm volatile("red.global.add.f32 [%0], %1;" ::"l"(p), "f"(v) : "memory");
 }
@@ -283,14 +289,16 @@ __device__ __forceinline__ void lookup_unit(const uint4 (&w)[Geom<MU, BT>::kVecs
 
 // Salient branch with row scales per group of GSV sub-vectors (grouped visit
 // order): after the GSV steps of slot a the lane has the whole contribution of
-// one (base, group) to its row and multiplies it by that group's row scale,
-// staged in shared memory in slot order.  One batch row (BT == 1).
+// one (base, group) kg = (a + lane/GSV) mod KG to its row and multiplies it by
+// that group's row scale, staged in shared memory as [kg][row of the CTA].
+// One batch row (BT == 1).
 template <int MU, int NB, int GSV, int HALF>
 __device__ __forceinline__ void lookup_unit_grouped(const uint4 (&w)[kSlabsPerWarp][Geom<MU, 1>::kVecs],
                                                     const Offsets<MU>& off, uint32_t tbase, uint32_t scale_row_off,
-                                                    float (&tot)[kSlabsPerWarp][1]) {
+                                                    int lane, float (&tot)[kSlabsPerWarp][1]) {
     constexpr int kStepsPerWord = 32 / MU;
     constexpr int KG = 32 / GSV;
+    const int m = lane / GSV;
 #pragma unroll
     for (int a = 0; a < KG; ++a) {
 #pragma unroll
@@ -302,8 +310,9 @@ __device__ __forceinline__ void lookup_unit_grouped(const uint4 (&w)[kSlabsPerWa
                 const int wi = q / kStepsPerWord;
                 g += lds_f32<HALF * 128>(tbase + off.addr(word_of(w[rs][wi / 4], wi % 4), q));
             }
+            const uint32_t kg = (uint32_t)((a + m) & (KG - 1));
             const float sc = __half2float(
-                smem_at<const __half>(scale_row_off + (uint32_t)(a * kRowsPerCta + rs * kLanes) * 2u));
+                smem_at<const __half>(scale_row_off + (kg * kRowsPerCta + (uint32_t)(rs * kLanes)) * 2u));
             tot[rs][0] = fmaf(sc, g, tot[rs][0]);
         }
     }
@@ -424,25 +433,82 @@ struct WeightRegs {
 };
 
 // Row scales of the grouped salient branch for unit u (a salient unit),
-// staged for parity `par` in slot order: entry [a][row] is the scale of the
-// (base, group) lane L = row % 32 completes at slot a.
+// staged for parity `par` as [kg][row of the CTA]: the KG (base, group)
+// pairs of the unit each hold 512 contiguous fp16 row scales, copied 8 rows
+// at a time by asynchronous 16-byte copies when M is a multiple of 8 and the
+// array is 16-byte aligned (element by element otherwise).  The caller waits
+// for the copies before the barrier that publishes them.
 template <int MU, int NB1, int GS1>
 __device__ __forceinline__ void stage_group_scales(const KernelArgs& a, int u, int rg, int tid, int par) {
     if constexpr (GS1 > 0) {
         constexpr int P = 32 / NB1, NG = P / GS1, KG = 32 / GS1;
+        constexpr int kChunks = kRowsPerCta / 8;
         const int ul = u - a.br[0].units;
         const __half* r = a.br[1].r;
         const int ng = a.br[1].ngroups;
-#pragma unroll 8
-        for (int e = tid; e < KG * kRowsPerCta; e += kThreads) {
-            const int slot = e / kRowsPerCta, lrow = e % kRowsPerCta;
-            const int kg = visit_group(lrow % kLanes, slot, GS1);
+        const int row0 = rg * kRowsPerCta;
+        const bool vec = (a.M % 8) == 0 && (reinterpret_cast<uintptr_t>(r) % 16) == 0;
+        const uint32_t dst0 = smem_base() + Geom<MU, 1>::kScaleOff + (uint32_t)(par * KG * kRowsPerCta) * 2u;
+#pragma unroll 2
+        for (int e = tid; e < KG * kChunks; e += kThreads) {
+            const int kg = e / kChunks, c = e % kChunks;
             const int k = kg / NG, gg = ul * NG + kg % NG;
-            const int row = rg * kRowsPerCta + lrow;
-            const __half v = (row < a.M && gg < ng) ? r[((int64_t)k * ng + gg) * a.M + row] : __float2half(0.f);
-            smem_at<__half>(Geom<MU, 1>::kScaleOff + (uint32_t)((par * KG + slot) * kRowsPerCta + lrow) * 2u) = v;
+            const int row = row0 + c * 8;
+            const uint32_t dst = dst0 + (uint32_t)(kg * kRowsPerCta + c * 8) * 2u;
+            const __half* src = r + ((int64_t)k * ng + gg) * a.M + row;
+            if (vec && gg < ng && row + 8 <= a.M) {
+                cp_async16(dst, src);
+            } else {
+#pragma unroll
+                for (int t = 0; t < 8; ++t) {
+                    const __half v = (gg < ng && row + t < a.M) ? src[t] : __float2half(0.f);
+                    asm volatile("st.shared.b16 [%0], %1;" ::"r"(dst + 2u * t), "h"(*reinterpret_cast<const unsigned short*>(&v)) : "memory");
+                }
+            }
         }
+        cp_async_commit();
     }
+}
+
+// Per-unit (block-wise) row scales of the lane's rows, kept as fp16 pairs in
+// a two-entry ring by unit parity like the packed words: the scales of unit u
+// are consumed at the end of its step and the entry is refilled with those of
+// unit u+2.  Units whose branch has per-row scales (or grouped salient scales)
+// leave the entry untouched.
+struct ScaleRing {
+    __half2 r[2][kSlabsPerWarp][2];
+};
+
+template <int MU, int NB0, int NB1, int GS1>
+__device__ __forceinline__ void load_block_scales(const KernelArgs& a, int u, int slab0, int lane,
+                                                  __half2 (&dst)[kSlabsPerWarp][2]) {
+    const bool br1 = NB1 > 0 && u >= a.br[0].units;
+    if (br1 && GS1 > 0) return;
+    const int rgroup = br1 ? a.br[1].rgroup : a.br[0].rgroup;
+    if (rgroup <= 0) return;
+    const __half* r = br1 ? a.br[1].r : a.br[0].r;
+    const int ng = br1 ? a.br[1].ngroups : a.br[0].ngroups;
+    const int nb = br1 ? (NB1 > 0 ? NB1 : 1) : NB0;
+    const int P = 32 / nb;
+    const int ul = br1 ? u - a.br[0].units : u;
+    const int g = (int)(((int64_t)ul * P * MU) / rgroup);
+#pragma unroll
+    for (int rs = 0; rs < kSlabsPerWarp; ++rs) {
+        const int i = (slab0 + rs) * kLanes + lane;
+        __half v[4];
+#pragma unroll
+        for (int ai = 0; ai < 4; ++ai) {
+            const int k = (ai + lane / P) % nb;
+            v[ai] = (ai < nb && i < a.M) ? r[((int64_t)k * ng + g) * a.M + i] : __float2half(0.f);
+        }
+        dst[rs][0] = __halves2half2(v[0], v[1]);
+        dst[rs][1] = __halves2half2(v[2], v[3]);
+    }
+}
+
+__device__ __forceinline__ float ring_scale(const __half2 (&e)[kSlabsPerWarp][2], int rs, int ai) {
+    const __half2 p = e[rs][ai / 2];
+    return __half2float((ai & 1) ? __high2half(p) : __low2half(p));
 }
 
 // One unit of branch BR: build its tables, form the next unit's products and
@@ -451,7 +517,7 @@ __device__ __forceinline__ void stage_group_scales(const KernelArgs& a, int u, i
 template <int MU, int BR, int NB, int HALF, int BT, int NB0, int NB1, int GS1>
 __device__ __forceinline__ void unit_step(const KernelArgs& a, int u, int u_end, int ul, int b0, int rg, int slab0,
                                           int warp, int lane, int tid, uint32_t sbase, const Offsets<MU>& off,
-                                          ProductPipe<BT>& pp, WeightRegs<MU, BT>& wb,
+                                          ProductPipe<BT>& pp, WeightRegs<MU, BT>& wb, ScaleRing& sr,
                                           float (&acc)[kSlabsPerWarp][BT][NB],
                                           float (&tot)[kSlabsPerWarp][BT]) {
     const BranchArgs& br = a.br[BR];
@@ -468,19 +534,7 @@ __device__ __forceinline__ void unit_step(const KernelArgs& a, int u, int u_end,
             pp.col2 = st.col;
         }
     }
-    float rsc[kSlabsPerWarp][NB];
-    if (!kGrouped && br.rgroup > 0) {
-        const int g = (int)(((int64_t)ul * P * MU) / br.rgroup);
-#pragma unroll
-        for (int rs = 0; rs < kSlabsPerWarp; ++rs) {
-            const int i = (slab0 + rs) * kLanes + lane;
-#pragma unroll
-            for (int ai = 0; ai < NB; ++ai) {
-                const int k = (ai + lane / P) % NB;
-                rsc[rs][ai] = i < a.M ? __half2float(br.r[((int64_t)k * br.ngroups + g) * a.M + i]) : 0.f;
-            }
-        }
-    }
+    if constexpr (GS1 > 0) cp_async_wait_all();  // this unit's staged salient scales
     __syncthreads();
     if constexpr (GS1 > 0) {
         // every warp is past the lookups of unit u-1, whose scale buffer this
@@ -498,7 +552,8 @@ __device__ __forceinline__ void unit_step(const KernelArgs& a, int u, int u_end,
         }
         const uint32_t scale_row_off = Geom<MU, 1>::kScaleOff +
             (uint32_t)((HALF * (32 / GS1)) * kRowsPerCta + (slab0 % kSlabsPerCta) * kLanes + lane) * 2u;
-        lookup_unit_grouped<MU, NB, GS1, HALF>(cur, off, sbase, scale_row_off, tot);
+        (void)P;
+        lookup_unit_grouped<MU, NB, GS1, HALF>(cur, off, sbase, scale_row_off, lane, tot);
     } else {
 #pragma unroll
         for (int rs = 0; rs < kSlabsPerWarp; ++rs) {
@@ -517,16 +572,17 @@ __device__ __forceinline__ void unit_step(const KernelArgs& a, int u, int u_end,
             for (int ai = 0; ai < NB; ++ai)
 #pragma unroll
                 for (int b = 0; b < BT; ++b) {
-                    tot[rs][b] = fmaf(rsc[rs][ai], acc[rs][b][ai], tot[rs][b]);
+                    tot[rs][b] = fmaf(ring_scale(sr.r[HALF], rs, ai), acc[rs][b][ai], tot[rs][b]);
                     acc[rs][b][ai] = 0.f;
                 }
     }
+    if (u + 2 < u_end) load_block_scales<MU, NB0, NB1, GS1>(a, u + 2, slab0, lane, sr.r[HALF]);
 }
 
 template <int MU, int BR, int NB, int BT, int NB0, int NB1, int GS1>
 __device__ __forceinline__ void run_branch(const KernelArgs& a, int u_lo, int u_hi, int u_end, int& v, int b0, int rg,
                                            int slab0, int warp, int lane, int tid, uint32_t sbase,
-                                           ProductPipe<BT>& pp, WeightRegs<MU, BT>& wb,
+                                           ProductPipe<BT>& pp, WeightRegs<MU, BT>& wb, ScaleRing& sr,
                                            float (&acc)[kSlabsPerWarp][BT][NB],
                                            float (&tot)[kSlabsPerWarp][BT]) {
     if (u_lo >= u_hi) return;
@@ -536,10 +592,10 @@ __device__ __forceinline__ void run_branch(const KernelArgs& a, int u_lo, int u_
     for (int u = u_lo; u < u_hi; ++u, ++v) {
         if (v & 1)
             unit_step<MU, BR, NB, 1, BT, NB0, NB1, GS1>(a, u, u_end, u - ubase, b0, rg, slab0, warp, lane, tid, sbase,
-                                                        off, pp, wb, acc, tot);
+                                                        off, pp, wb, sr, acc, tot);
         else
             unit_step<MU, BR, NB, 0, BT, NB0, NB1, GS1>(a, u, u_end, u - ubase, b0, rg, slab0, warp, lane, tid, sbase,
-                                                        off, pp, wb, acc, tot);
+                                                        off, pp, wb, sr, acc, tot);
     }
 }
 
@@ -596,6 +652,7 @@ __global__ void __launch_bounds__(kThreads, min_blocks<BT>()) fluxbin_lut_kernel
     asm volatile("griddepcontrol.launch_dependents;");
 
     WeightRegs<MU, BT> wb;
+    ScaleRing sr;
     float sc0[kSlabsPerWarp][NB0], sc1[kSlabsPerWarp][NB1E];
     SlotStatic st0{0.f, -1}, st1{0.f, -1}, st2{0.f, -1};
     const bool slot_owner = tid < G::kSlots;
@@ -608,6 +665,8 @@ __global__ void __launch_bounds__(kThreads, min_blocks<BT>()) fluxbin_lut_kernel
                 for (int rs = 0; rs < kSlabsPerWarp; ++rs)
                     load_unit_slab<MU, BT>(a, u_begin + d, slab0 + rs, lane, wb.w[d][rs]);
             }
+        if (u_begin < u_end) load_block_scales<MU, NB0, NB1, GS1>(a, u_begin, slab0, lane, sr.r[0]);
+        if (u_begin + 1 < u_end) load_block_scales<MU, NB0, NB1, GS1>(a, u_begin + 1, slab0, lane, sr.r[1]);
         fetch_row_scales<NB0>(a, a.br[0], slab0, lane, sc0);
         if constexpr (NB1 > 0) fetch_row_scales<NB1>(a, a.br[1], slab0, lane, sc1);
         if (slot_owner) {
@@ -630,6 +689,7 @@ __global__ void __launch_bounds__(kThreads, min_blocks<BT>()) fluxbin_lut_kernel
     }
     if constexpr (GS1 > 0) {
         if (u_begin < u_end && u_begin >= U0) stage_group_scales<MU, NB1, GS1>(a, u_begin, rg, tid, 0);
+        cp_async_wait_all();
     }
     if (slot_owner) {
         pp.c1 = st1.c;
@@ -654,10 +714,10 @@ __global__ void __launch_bounds__(kThreads, min_blocks<BT>()) fluxbin_lut_kernel
 
     int v = 0;
     run_branch<MU, 0, NB0, BT, NB0, NB1, GS1>(a, u_begin, min(u_end, U0), u_end, v, b0, rg, slab0, warp, lane, tid,
-                                              sbase, pp, wb, acc0, tot);
+                                              sbase, pp, wb, sr, acc0, tot);
     if constexpr (NB1 > 0)
         run_branch<MU, 1, NB1, BT, NB0, NB1, GS1>(a, max(u_begin, U0), u_end, u_end, v, b0, rg, slab0, warp, lane, tid,
-                                                  sbase, pp, wb, acc1, tot);
+                                                  sbase, pp, wb, sr, acc1, tot);
 
     // Row scales (per-row case; the block-wise case was applied per unit).
 #pragma unroll

@@ -7,43 +7,80 @@
 // weights are streamed as compressed uint32 words, never rebuilt as floats.
 #include <string.h>
 
+#include <algorithm>
+#include <thread>
+#include <vector>
+
 #include "fluxbin_host.h"
 
 using namespace fluxbin;
 
 namespace {
 
+// Packs rows [i0, i1) of one branch.  Every row writes only the words of its
+// own lane (the layout interleaves the 32 rows of a slab word by word), so
+// disjoint row ranges can be packed concurrently.
+int pack_rows(const int8_t* signs, int64_t M, int64_t ncols, int nb, int mu, const uint8_t* qtab, int64_t i0,
+              int64_t i1, uint32_t* words) {
+    const int P = subvecs_per_unit(nb);
+    const int64_t U = branch_units(ncols, nb, mu);
+    const int64_t cw = chunk_words(mu);
+    const int64_t nsub = (ncols + mu - 1) / mu;
+    for (int k = 0; k < nb; ++k) {
+        for (int64_t i = i0; i < i1; ++i) {
+            const int8_t* row = signs + ((int64_t)k * M + i) * ncols;
+            const int L = (int)(i % kLanes);
+            const uint8_t* qrow = qtab + ((size_t)L * nb + k) * P;
+            uint32_t* slab = words + (i / kLanes) * U * cw + (int64_t)L * 4;
+            int bad = 0;
+            for (int64_t jg = 0; jg < nsub; ++jg) {
+                const int64_t n0 = jg * mu;
+                const int len = (int)std::min<int64_t>(mu, ncols - n0);
+                uint32_t pat = 0;
+                for (int t = 0; t < len; ++t) {
+                    const int8_t v = row[n0 + t];
+                    pat |= (uint32_t)(v == 1) << t;
+                    bad |= (v != 1) & (v != -1);
+                }
+                const int pos = qrow[jg % P] * mu;
+                slab[(jg / P) * cw + (int64_t)(pos / 128) * kLanes * 4 + (pos / 32) % 4] |= pat << (pos % 32);
+            }
+            if (bad) return FLUXBIN_ERR_BAD_SHAPE;
+        }
+    }
+    return FLUXBIN_OK;
+}
+
 // Packs one branch: signs [nb][M][ncols] (+-1) -> words (device layout);
 // gsv selects the visit order (see fluxbin_layout.h).
 int pack_branch(const int8_t* signs, int64_t M, int64_t ncols, int nb, int mu, int gsv, uint32_t* words) {
     const int P = subvecs_per_unit(nb);
-    const int64_t U = branch_units(ncols, nb, mu);
     const int64_t total = branch_words(M, ncols, nb, mu);
     memset(words, 0, (size_t)total * sizeof(uint32_t));
-    const int64_t nsub = (ncols + mu - 1) / mu;
-    for (int k = 0; k < nb; ++k) {
-        for (int64_t i = 0; i < M; ++i) {
-            const int8_t* row = signs + ((int64_t)k * M + i) * ncols;
-            const int64_t s = i / kLanes;
-            const int L = (int)(i % kLanes);
-            for (int64_t jg = 0; jg < nsub; ++jg) {
-                uint32_t pat = 0;
-                const int64_t n0 = jg * mu;
-                for (int t = 0; t < mu && n0 + t < ncols; ++t) {
-                    const int8_t v = row[n0 + t];
-                    if (v == 1) pat |= 1u << t;
-                    else if (v != -1) return FLUXBIN_ERR_BAD_SHAPE;
-                }
-                if (!pat) continue;
-                const int64_t u = jg / P;
-                const int j = (int)(jg % P);
-                const int q = visit_step(L, k, j, nb, gsv);
-                const int pos = q * mu;
-                const int64_t w = (s * U + u) * chunk_words(mu) + ((int64_t)(pos / 128) * kLanes + L) * 4 + (pos / 32) % 4;
-                words[w] |= pat << (pos % 32);
-            }
-        }
+    std::vector<uint8_t> qtab((size_t)kLanes * nb * P);
+    for (int L = 0; L < kLanes; ++L)
+        for (int k = 0; k < nb; ++k)
+            for (int j = 0; j < P; ++j) qtab[((size_t)L * nb + k) * P + j] = (uint8_t)visit_step(L, k, j, nb, gsv);
+    const int64_t slabs = (M + kLanes - 1) / kLanes;
+    const int64_t work = M * ncols * nb;
+    unsigned nt = std::max(1u, std::thread::hardware_concurrency());
+    if (nt > 32) nt = 32;
+    if (work < (int64_t)1 << 22 || slabs < 2) nt = 1;
+    if ((int64_t)nt > slabs) nt = (unsigned)slabs;
+    std::vector<int> status(nt, FLUXBIN_OK);
+    auto job = [&](unsigned t) {
+        const int64_t s0 = slabs * t / nt, s1 = slabs * (t + 1) / nt;
+        status[t] = pack_rows(signs, M, ncols, nb, mu, qtab.data(), s0 * kLanes, std::min(M, s1 * kLanes), words);
+    };
+    if (nt == 1) {
+        job(0);
+    } else {
+        std::vector<std::thread> th;
+        for (unsigned t = 0; t < nt; ++t) th.emplace_back(job, t);
+        for (auto& x : th) x.join();
     }
+    for (int st : status)
+        if (st != FLUXBIN_OK) return st;
     return FLUXBIN_OK;
 }
 

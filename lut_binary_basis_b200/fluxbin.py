@@ -175,6 +175,16 @@ def fluxbin_linear_static_scratch(desc: LayerDesc, words, r, c, swords, rs, cs, 
                                                _stream(stream)), "fluxbin_linear_static_scratch")
 
 
+def pack_host(layer) -> dict:
+    """Pack a host layer (``LayerData``) with the library's packer: the host
+    arrays a device layer is made of (no CUDA involved)."""
+    desc = LayerDesc.of(layer.spec)
+    words, swords = fluxbin_pack(desc, layer.signs, layer.sal_signs if desc.Ks else None,
+                                 layer.sal_idx if desc.Ks else None)
+    return {"desc": desc, "words": words, "r": layer.r, "c": layer.c, "swords": swords, "rs": layer.rs,
+            "cs": layer.cs, "idx": layer.sal_idx.astype(np.int32)}
+
+
 @dataclasses.dataclass
 class DeviceLayer:
     """One packed layer resident on a CUDA device (torch owns the memory)."""
@@ -191,19 +201,22 @@ class DeviceLayer:
     @classmethod
     def from_host(cls, layer, device="cuda") -> "DeviceLayer":
         """Pack a host layer (``LayerData``) with the library's packer and copy it to ``device``."""
+        return cls.from_packed(pack_host(layer), device)
+
+    @classmethod
+    def from_packed(cls, packed: dict, device="cuda") -> "DeviceLayer":
+        """Copy the arrays of ``pack_host`` to ``device``."""
         import torch
-        desc = LayerDesc.of(layer.spec)
-        words, swords = fluxbin_pack(desc, layer.signs, layer.sal_signs if desc.Ks else None,
-                                     layer.sal_idx if desc.Ks else None)
 
         def dev(a, dtype):
             a = np.ascontiguousarray(a)
             t = torch.from_numpy(a.view(dtype) if a.size else np.zeros(1, dtype))
             return t.to(device)
 
-        return cls(desc, dev(words, np.int32), dev(layer.r, np.float16), dev(layer.c, np.float16),
-                   dev(swords, np.int32), dev(layer.rs, np.float16), dev(layer.cs, np.float16),
-                   dev(layer.sal_idx.astype(np.int32), np.int32))
+        p = packed
+        return cls(p["desc"], dev(p["words"], np.int32), dev(p["r"], np.float16), dev(p["c"], np.float16),
+                   dev(p["swords"], np.int32), dev(p["rs"], np.float16), dev(p["cs"], np.float16),
+                   dev(p["idx"], np.int32))
 
     def linear(self, x, y, flags: int = FLAG_Y_FP32, workspace=None, stream=None) -> None:
         B = x.shape[0] if x.dim() == 2 else 1

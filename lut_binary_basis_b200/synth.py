@@ -87,10 +87,16 @@ def _rng(key: Sequence[int]) -> Dict[str, np.random.Generator]:
 
 
 def _signs(g: np.random.Generator, shape) -> np.ndarray:
-    bits = g.integers(0, 2, size=shape, dtype=np.int8)
-    bits <<= 1
-    bits -= 1
-    return bits
+    """iid fair +-1 signs: the bits of the generator's raw 64-bit output, each
+    byte spread to eight sign bytes by one multiply (bit t -> byte 7-t)."""
+    n = int(np.prod(shape))
+    raw = g.bit_generator.random_raw((n + 63) // 64).astype(np.uint64)
+    byt = raw.view(np.uint8)[: (n + 7) // 8].astype(np.uint64)
+    spread = ((byt * np.uint64(0x8040201008040201)) & np.uint64(0x8080808080808080)) >> np.uint64(7)
+    s = spread.view(np.int8)[:n]
+    s = s * np.int8(2)
+    s -= np.int8(1)
+    return s.reshape(shape)
 
 
 def _lognormal_fp16(g: np.random.Generator, shape, sigma: float = 0.3) -> np.ndarray:

@@ -218,6 +218,9 @@ FULL = [
     (synth.layers_70b_mlp(8)[1], [16], 3),
     (synth.layers_70b_mlp(4)[0], [16], 3),
     (synth.layers_70b_mlp(4)[1], [1], 3),
+    (synth.layers_7b_stack_linears()[0], [1], 4),   # q: 2.75-bit, block-wise and grouped salient scales
+    (synth.layers_7b_stack_linears()[4], [1], 4),   # gate
+    (synth.layers_7b_stack_linears()[6], [1], 4),   # down
 ]
 
 
