@@ -133,6 +133,24 @@ typedef struct fluxbin_layer_desc {
                                          still running before this call writes the layer's packed
                                          words.  x, y, scales and workspace are always read only
                                          after the preceding kernel has completed. */
+#define FLUXBIN_FLAG_PATH_LUT     8u  /* always use the LUT path */
+#define FLUXBIN_FLAG_PATH_TC      16u /* always use the tensor-core path (UNSUPPORTED when the layer
+                                         does not qualify, WORKSPACE without a workspace) */
+/*
+ * Two execution paths compute the same layer.  The LUT path builds the 2^mu
+ * signed partial sums of every activation sub-vector in shared memory and
+ * looks them up with the packed bit patterns (FluxBin summary, Section 3
+ * "LUT-Based GEMV Kernel").  The tensor-core path, for larger batches, expands
+ * the +-1 signs of each unit into fp16 in shared memory only and contracts them
+ * with the fp16 products c (.) x on the tensor cores (tcgen05.mma), fp32
+ * accumulation in tensor memory, row scales applied to the accumulators (the
+ * LUT Tensor Core notes, Section 2.2, read LUT-based mixed-precision GEMM as a
+ * GEMM with one low-bit operand).  It needs mu == 8, per-row scales
+ * (row_scale_group == 0 and sal_scale_group == 0) and a workspace; it is taken
+ * by default when B >= 8 and the layer qualifies, and may be forced either way
+ * with the flags above.  Its products are rounded to fp16 before the
+ * contraction (relative error below 2^-11 per product).
+ */
 
 /* Human-readable name of a status code (static storage, never NULL). */
 const char* fluxbin_status_string(int status);
@@ -140,6 +158,14 @@ const char* fluxbin_status_string(int status);
 /* Name and description of the last CUDA failure (FLUXBIN_ERR_CUDA) seen by a
  * call on this host thread; "" if none.  Thread-local storage, never NULL. */
 const char* fluxbin_last_error(void);
+
+/*
+ * Device-side status of the current device: bit 0 is set when a tensor-core
+ * launch gave up waiting for its own tensor-core operations (never expected;
+ * its outputs are then NaN).  Reads and clears the flags; synchronises with
+ * the device.  Errors: INVALID_ARG (null output), CUDA.
+ */
+int fluxbin_device_status(uint32_t* out_flags);
 
 /* Library version: major*10000 + minor*100 + patch. */
 int fluxbin_version(void);

@@ -22,7 +22,7 @@ NVCC_FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-Xcompil
               "--expt-relaxed-constexpr", "-I", os.path.join(ROOT, "include")] + ARCH
 CXX_FLAGS = ["-O2", "-std=c++17", "-fPIC", "-Wall", "-I", os.path.join(ROOT, "include")]
 
-CU_SOURCES = ["fluxbin_api.cu", "fluxbin_inst_mu8.cu", "fluxbin_inst_mu4.cu"]
+CU_SOURCES = ["fluxbin_api.cu", "fluxbin_inst_mu8.cu", "fluxbin_inst_mu4.cu", "fluxbin_inst_tc.cu"]
 CXX_SOURCES = ["fluxbin_pack.cpp"]
 
 

@@ -9,12 +9,22 @@
 
 #include "fluxbin_host.h"
 #include "fluxbin_kernel.cuh"
+#include "fluxbin_tc.cuh"
+
+// Set by the tensor-core kernel when one of its bounded waits gives up; read
+// and cleared by fluxbin_device_status.  One copy per device.
+static __device__ unsigned int g_fluxbin_device_error;
 
 namespace fluxbin {
 
 using KernelFn = void (*)(KernelArgs);
 KernelFn select_kernel_mu8(int nb0, int nb1, int bt, int gs1);
 KernelFn select_kernel_mu4(int nb0, int nb1, int bt, int gs1);
+using TcKernelFn = void (*)(TcArgs);
+TcKernelFn select_tc_kernel(int nb0, int nb1);
+
+// Smallest batch the automatic path choice sends to the tensor cores.
+constexpr int kTcMinBatch = 8;
 
 namespace {
 
@@ -177,9 +187,119 @@ Plan make_plan(KernelFn fn, int dev, int mu, int bt, int gs1, int64_t Ms, int64_
     return p;
 }
 
+constexpr int kMaxDevicesTc = 64;
+std::mutex g_tc_mu;
+std::unordered_map<uint64_t, bool> g_tc_func;
+unsigned int* g_err_addr[kMaxDevicesTc] = {};
+
+int device_error_address(int dev, unsigned int** out) {
+    if (dev < 0 || dev >= kMaxDevicesTc) return FLUXBIN_ERR_CUDA;
+    if (!g_err_addr[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_fluxbin_device_error) != cudaSuccess || !p) {
+            (void)cudaGetLastError();
+            return FLUXBIN_ERR_CUDA;
+        }
+        g_err_addr[dev] = static_cast<unsigned int*>(p);
+    }
+    *out = g_err_addr[dev];
+    return FLUXBIN_OK;
+}
+
+// The layer on the tensor cores (fluxbin_tc.cuh): per-row scales, mu = 8,
+// 1 <= B <= 16, a workspace always (the split of a tile's units is reduced
+// through it).  Items (128-row tile, unit range) run on a persistent grid of
+// one CTA per SM; the unit ranges are split so that there are about four
+// items per SM.
+int run_tc(int32_t M, int32_t N, const BranchIn& g, const BranchIn* s, int nb1, const uint16_t* d_x, int32_t B,
+           void* d_y, uint32_t flags, void* ws, size_t ws_bytes, void* stream) {
+    const size_t need = workspace_bytes_for(M, B);
+    if (!ws || ws_bytes < need) return FLUXBIN_ERR_WORKSPACE;
+    if (!aligned(ws, 16)) return FLUXBIN_ERR_MISALIGNED;
+    TcKernelFn fn = select_tc_kernel(g.nb, nb1);
+    if (!fn) return FLUXBIN_ERR_UNSUPPORTED;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return FLUXBIN_ERR_CUDA;
+    DeviceInfo di;
+    unsigned int* err = nullptr;
+    {
+        std::lock_guard<std::mutex> lock(g_mu);
+        int st = device_info(dev, &di);
+        if (st != FLUXBIN_OK) return st;
+    }
+    {
+        std::lock_guard<std::mutex> lock(g_tc_mu);
+        int st = device_error_address(dev, &err);
+        if (st != FLUXBIN_OK) return st;
+        const uint64_t key = (reinterpret_cast<uint64_t>(fn) << 8) ^ (uint64_t)dev;
+        if (g_tc_func.find(key) == g_tc_func.end()) {
+            cudaFuncAttributes fa;
+            cudaError_t e = cudaFuncGetAttributes(&fa, fn);
+            if (e != cudaSuccess) return cuda_fail(e);
+            if ((size_t)di.max_smem < (size_t)kTcSmemBytes + fa.sharedSizeBytes) return FLUXBIN_ERR_SMEM_BUDGET;
+            int blocks = 0;
+            if ((e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, kTcSmemBytes)) !=
+                    cudaSuccess ||
+                (e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&blocks, fn, kTcThreads + 32, kTcSmemBytes)) !=
+                    cudaSuccess)
+                return cuda_fail(e);
+            if (blocks < 1) return FLUXBIN_ERR_SMEM_BUDGET;
+            g_tc_func.emplace(key, true);
+        }
+    }
+    TcArgs a = {};
+    const BranchIn* in[2] = {&g, nb1 ? s : nullptr};
+    for (int q = 0; q < 2; ++q) {
+        BranchArgs& o = a.br[q];
+        if (!in[q] || in[q]->ncols == 0) continue;
+        o.words = reinterpret_cast<const uint4*>(in[q]->words);
+        o.r = reinterpret_cast<const __half*>(in[q]->r);
+        o.c = reinterpret_cast<const __half*>(in[q]->c);
+        o.gather = in[q]->gather;
+        o.ncols = in[q]->ncols;
+        o.units = (int32_t)branch_units(in[q]->ncols, in[q]->nb, 8);
+    }
+    const int64_t U = (int64_t)a.br[0].units + a.br[1].units;
+    a.x = reinterpret_cast<const __half*>(d_x);
+    a.y = d_y;
+    a.M = M;
+    a.N = N;
+    a.B = B;
+    a.Ms = (int32_t)row_slabs(M);
+    a.Mp = a.Ms * kLanes;
+    a.n_rt = (M + kTcRows - 1) / kTcRows;
+    int64_t ks = (4 * (int64_t)di.sm_count + a.n_rt - 1) / a.n_rt;
+    if (ks > U) ks = U;
+    if (ks < 1) ks = 1;
+    a.n_ks = (int32_t)ks;
+    a.n_items = a.n_rt * a.n_ks;
+    a.flags = flags;
+    const size_t acc = (((size_t)B * a.Mp * sizeof(float)) + 255) & ~(size_t)255;
+    a.ws_acc = static_cast<float*>(ws);
+    a.ws_cnt = reinterpret_cast<unsigned int*>(static_cast<char*>(ws) + acc);
+    a.err = err;
+    a.vec_x = (N % 8 == 0 && aligned(d_x, 16) && aligned(g.c, 16)) ? 1 : 0;
+
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(a.n_items < di.sm_count ? a.n_items : di.sm_count));
+    cfg.blockDim = dim3(kTcThreads + 32);   // 16 worker warps and the MMA-issuing warp
+    cfg.dynamicSmemBytes = kTcSmemBytes;
+    cfg.stream = static_cast<cudaStream_t>(stream);
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t le = cudaLaunchKernelEx(&cfg, fn, a);
+    if (le != cudaSuccess) return cuda_fail(le);
+    return FLUXBIN_OK;
+}
+
 int run(int32_t M, int32_t N, int mu, const BranchIn& g, const BranchIn* s, const uint16_t* d_x, int32_t B,
         void* d_y, uint32_t flags, void* ws, size_t ws_bytes, void* stream) {
-    if (flags & ~(kFlagAccumulate | kFlagYFp32 | kFlagEarlyWeights)) return FLUXBIN_ERR_INVALID_ARG;
+    if (flags & ~(kFlagAccumulate | kFlagYFp32 | kFlagEarlyWeights | kFlagPathLut | kFlagPathTc))
+        return FLUXBIN_ERR_INVALID_ARG;
+    if ((flags & kFlagPathLut) && (flags & kFlagPathTc)) return FLUXBIN_ERR_INVALID_ARG;
     if (B < 0 || B > kMaxBatch) return B < 0 ? FLUXBIN_ERR_BAD_SHAPE : FLUXBIN_ERR_UNSUPPORTED;
     if (M == 0 || B == 0) return FLUXBIN_OK;
     if (!d_y || (N > 0 && !d_x)) return FLUXBIN_ERR_INVALID_ARG;
@@ -194,6 +314,13 @@ int run(int32_t M, int32_t N, int mu, const BranchIn& g, const BranchIn* s, cons
         if (!aligned(b->r, 2) || !aligned(b->c, 2) || !aligned(b->gather, 4)) return FLUXBIN_ERR_MISALIGNED;
     }
     const int nb1 = (s && s->ncols > 0) ? s->nb : 0;
+    // the tensor-core path: per-row scales, mu = 8, a batch large enough for
+    // the contraction to pay (or asked for explicitly)
+    const bool tc_fits = mu == 8 && g.rgroup == 0 && (!nb1 || s->rgroup == 0);
+    if ((flags & kFlagPathTc) && !tc_fits) return FLUXBIN_ERR_UNSUPPORTED;
+    if ((flags & kFlagPathTc) ||
+        (!(flags & kFlagPathLut) && tc_fits && B >= kTcMinBatch && ws && ws_bytes >= workspace_bytes_for(M, B)))
+        return run_tc(M, N, g, s, nb1, d_x, B, d_y, flags & ~(kFlagPathLut | kFlagPathTc), ws, ws_bytes, stream);
     // salient row scales finer than a unit: grouped visit order, one batch row per CTA
     const int gs1 = (nb1 && s->rgroup > 0 && s->rgroup < unit_cols(nb1, mu)) ? s->rgroup / mu : 0;
     const int bt = gs1 ? 1 : batch_tile(mu, B);
@@ -280,6 +407,24 @@ using namespace fluxbin;
 extern "C" {
 
 const char* fluxbin_last_error(void) { return g_last_error; }
+
+int fluxbin_device_status(uint32_t* out_flags) {
+    if (!out_flags) return FLUXBIN_ERR_INVALID_ARG;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return FLUXBIN_ERR_CUDA;
+    unsigned int* err = nullptr;
+    {
+        std::lock_guard<std::mutex> lock(g_tc_mu);
+        const int st = device_error_address(dev, &err);
+        if (st != FLUXBIN_OK) return st;
+    }
+    unsigned int v = 0;
+    cudaError_t e = cudaMemcpy(&v, err, sizeof(v), cudaMemcpyDeviceToHost);
+    if (e == cudaSuccess && v) e = cudaMemset(err, 0, sizeof(v));
+    if (e != cudaSuccess) return cuda_fail(e);
+    *out_flags = v;
+    return FLUXBIN_OK;
+}
 
 int fluxbin_lut_gemv(int32_t M, int32_t N, int32_t ncols, int32_t nbases, int32_t mu, int32_t row_scale_group,
                      const uint32_t* d_words, const uint16_t* d_r, const uint16_t* d_c, const int32_t* d_gather,

@@ -47,7 +47,10 @@ inline size_t workspace_bytes_for(int64_t M, int64_t B) {
     const int64_t n_rg = (row_slabs(M) + kSlabsPerCta - 1) / kSlabsPerCta;
     size_t acc = (size_t)(B * Mp) * sizeof(float);
     acc = (acc + 255) & ~(size_t)255;
-    size_t cnt = (size_t)(n_rg * B) * sizeof(unsigned int);
+    // arrival counters: one per 512-row group and batch chunk (LUT path) or
+    // one per 128-row tile (tensor-core path), whichever is more
+    const int64_t n_rt = (row_slabs(M) + 3) / 4;
+    size_t cnt = (size_t)(n_rg * B > n_rt ? n_rg * B : n_rt) * sizeof(unsigned int);
     return acc + ((cnt + 255) & ~(size_t)255);
 }
 

@@ -85,6 +85,8 @@ struct KernelArgs {
 constexpr uint32_t kFlagAccumulate = 1u;
 constexpr uint32_t kFlagYFp32 = 2u;
 constexpr uint32_t kFlagEarlyWeights = 4u;
+constexpr uint32_t kFlagPathLut = 8u;
+constexpr uint32_t kFlagPathTc = 16u;
 
 template <int MU, int BT>
 struct Geom {

@@ -20,6 +20,8 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libfluxbin.
 FLAG_ACCUMULATE = 1
 FLAG_Y_FP32 = 2
 FLAG_EARLY_WEIGHTS = 4
+FLAG_PATH_LUT = 8
+FLAG_PATH_TC = 16
 
 STATUS = {0: "FLUXBIN_OK", -1: "FLUXBIN_ERR_INVALID_ARG", -2: "FLUXBIN_ERR_BAD_SHAPE",
           -3: "FLUXBIN_ERR_MISALIGNED", -4: "FLUXBIN_ERR_UNSUPPORTED", -5: "FLUXBIN_ERR_SMEM_BUDGET",
@@ -73,8 +75,9 @@ def lib():
             L.fluxbin_lut_gemv.argtypes = [i32, i32, i32, i32, i32, i32, P, P, P, P, P, i32, P, u32, P, sz, P]
             L.fluxbin_linear.argtypes = [P, P, P, P, P, P, P, P, P, i32, P, u32, P, sz, P]
             L.fluxbin_linear_static_scratch.argtypes = [P, P, P, P, P, P, P, P, P, i32, P, u32, P]
+            L.fluxbin_device_status.argtypes = [ctypes.POINTER(u32)]
             for f in ("fluxbin_packed_sizes", "fluxbin_pack", "fluxbin_workspace_bytes", "fluxbin_lut_gemv",
-                      "fluxbin_linear", "fluxbin_linear_static_scratch"):
+                      "fluxbin_linear", "fluxbin_linear_static_scratch", "fluxbin_device_status"):
                 getattr(L, f).restype = ctypes.c_int
             _lib = L
     return _lib
@@ -91,6 +94,13 @@ def fluxbin_status_string(status: int) -> str:
 
 def fluxbin_last_error() -> str:
     return lib().fluxbin_last_error().decode()
+
+
+def fluxbin_device_status() -> int:
+    """Device-side status flags of the current device (read and cleared)."""
+    v = ctypes.c_uint32(0)
+    _check(lib().fluxbin_device_status(ctypes.byref(v)), "fluxbin_device_status")
+    return int(v.value)
 
 
 def fluxbin_version() -> int:
