@@ -145,7 +145,7 @@ typedef struct fluxbin_layer_desc {
  * with the fp16 products c (.) x on the tensor cores (tcgen05.mma), fp32
  * accumulation in tensor memory, row scales applied to the accumulators (the
  * LUT Tensor Core notes, Section 2.2, read LUT-based mixed-precision GEMM as a
- * GEMM with one low-bit operand).  It needs mu == 8, per-row scales
+ * GEMM with one low-bit operand).  It needs mu == 4 or 8, per-row scales
  * (row_scale_group == 0 and sal_scale_group == 0) and a workspace; it is taken
  * by default when B >= 8 and the layer qualifies, and may be forced either way
  * with the flags above.  Its products are rounded to fp16 before the

@@ -21,7 +21,7 @@ using KernelFn = void (*)(KernelArgs);
 KernelFn select_kernel_mu8(int nb0, int nb1, int bt, int gs1);
 KernelFn select_kernel_mu4(int nb0, int nb1, int bt, int gs1);
 using TcKernelFn = void (*)(TcArgs);
-TcKernelFn select_tc_kernel(int nb0, int nb1);
+TcKernelFn select_tc_kernel(int mu, int nb0, int nb1);
 
 // Smallest batch the automatic path choice sends to the tensor cores.
 constexpr int kTcMinBatch = 8;
@@ -206,17 +206,17 @@ int device_error_address(int dev, unsigned int** out) {
     return FLUXBIN_OK;
 }
 
-// The layer on the tensor cores (fluxbin_tc.cuh): per-row scales, mu = 8,
+// The layer on the tensor cores (fluxbin_tc.cuh): per-row scales, mu = 4 or 8,
 // 1 <= B <= 16, a workspace always (the split of a tile's units is reduced
 // through it).  Items (128-row tile, unit range) run on a persistent grid of
 // one CTA per SM; the unit ranges are split so that there are about four
 // items per SM.
-int run_tc(int32_t M, int32_t N, const BranchIn& g, const BranchIn* s, int nb1, const uint16_t* d_x, int32_t B,
+int run_tc(int32_t M, int32_t N, int mu, const BranchIn& g, const BranchIn* s, int nb1, const uint16_t* d_x, int32_t B,
            void* d_y, uint32_t flags, void* ws, size_t ws_bytes, void* stream) {
     const size_t need = workspace_bytes_for(M, B);
     if (!ws || ws_bytes < need) return FLUXBIN_ERR_WORKSPACE;
     if (!aligned(ws, 16)) return FLUXBIN_ERR_MISALIGNED;
-    TcKernelFn fn = select_tc_kernel(g.nb, nb1);
+    TcKernelFn fn = select_tc_kernel(mu, g.nb, nb1);
     if (!fn) return FLUXBIN_ERR_UNSUPPORTED;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return FLUXBIN_ERR_CUDA;
@@ -257,7 +257,7 @@ int run_tc(int32_t M, int32_t N, const BranchIn& g, const BranchIn* s, int nb1, 
         o.c = reinterpret_cast<const __half*>(in[q]->c);
         o.gather = in[q]->gather;
         o.ncols = in[q]->ncols;
-        o.units = (int32_t)branch_units(in[q]->ncols, in[q]->nb, 8);
+        o.units = (int32_t)branch_units(in[q]->ncols, in[q]->nb, mu);
     }
     const int64_t U = (int64_t)a.br[0].units + a.br[1].units;
     a.x = reinterpret_cast<const __half*>(d_x);
@@ -316,11 +316,11 @@ int run(int32_t M, int32_t N, int mu, const BranchIn& g, const BranchIn* s, cons
     const int nb1 = (s && s->ncols > 0) ? s->nb : 0;
     // the tensor-core path: per-row scales, mu = 8, a batch large enough for
     // the contraction to pay (or asked for explicitly)
-    const bool tc_fits = mu == 8 && g.rgroup == 0 && (!nb1 || s->rgroup == 0);
+    const bool tc_fits = (mu == 8 || mu == 4) && g.rgroup == 0 && (!nb1 || s->rgroup == 0);
     if ((flags & kFlagPathTc) && !tc_fits) return FLUXBIN_ERR_UNSUPPORTED;
     if ((flags & kFlagPathTc) ||
         (!(flags & kFlagPathLut) && tc_fits && B >= kTcMinBatch && ws && ws_bytes >= workspace_bytes_for(M, B)))
-        return run_tc(M, N, g, s, nb1, d_x, B, d_y, flags & ~(kFlagPathLut | kFlagPathTc), ws, ws_bytes, stream);
+        return run_tc(M, N, mu, g, s, nb1, d_x, B, d_y, flags & ~(kFlagPathLut | kFlagPathTc), ws, ws_bytes, stream);
     // salient row scales finer than a unit: grouped visit order, one batch row per CTA
     const int gs1 = (nb1 && s->rgroup > 0 && s->rgroup < unit_cols(nb1, mu)) ? s->rgroup / mu : 0;
     const int bt = gs1 ? 1 : batch_tile(mu, B);

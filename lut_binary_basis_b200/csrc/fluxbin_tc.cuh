@@ -112,24 +112,30 @@ __device__ __forceinline__ uint64_t tc_smem_desc_sw128(uint32_t addr) {
            (2ull << 61);
 }
 
-// Byte offset of the 16-byte chunk of sub-vector j (base k) of row r in an
-// operand buffer with `groups` 8-row groups per 64-column block.
-template <int NB>
-__device__ __forceinline__ uint32_t sw128_chunk(int k, int j, int r, int groups) {
-    constexpr int P = 32 / NB;
-    return (uint32_t)((((k * (P / 8) + (j >> 3)) * groups + (r >> 3)) << 10) + ((r & 7) << 7) +
-                      ((((j & 7) ^ (r & 7))) << 4));
-}
-
 // Instruction descriptor: fp32 accumulator, fp16 A and B, both K-major,
 // N = 16, M = 128.
 constexpr uint32_t kTcIdesc = (1u << 4) | ((uint32_t)(kTcN >> 3) << 17) | ((uint32_t)(kTcRows >> 4) << 24);
 
-// The 16 MMAs of one unit (nb bases x P/2 K steps of 16): the descriptors of
-// the unit's A and B buffers are built once; each MMA adds its operands'
-// offsets (in 16-byte units) to the start-address field.  Accumulator k of
-// the branch lives at TMEM column (acc0 + k) * 16.
-template <int NB>
+// A unit's K axis concatenates its bases: sub-vector j of base k covers
+// K = (k*P + j)*MU .. +MU-1.  Byte offset of element block (k, j) of row r in
+// an operand buffer with `groups` 8-row groups per 64-column atom: atom
+// ck/8, 16-byte chunk ck%8 (xor-swizzled with r%8), ck = (k*P + j)*MU/8, and
+// for MU = 4 the half (k*P + j)%2 of that chunk.
+template <int MU, int NB>
+__device__ __forceinline__ uint32_t sw128_block(int k, int j, int r, int groups) {
+    constexpr int P = 32 / NB;
+    const int kj = k * P + j;
+    const int ck = MU == 8 ? kj : (kj >> 1);
+    const int half = MU == 8 ? 0 : (kj & 1);
+    return (uint32_t)((((ck >> 3) * groups + (r >> 3)) << 10) + ((r & 7) << 7) + (((ck & 7) ^ (r & 7)) << 4) +
+                      (half << 3));
+}
+
+// The MMAs of one unit (nb bases x P*MU/16 K steps of 16; 16 for MU = 8, 8
+// for MU = 4): the descriptors of the unit's A and B buffers are built once;
+// each MMA adds its operands' offsets (in 16-byte units) to the start-address
+// field.  Accumulator k of the branch lives at TMEM column (acc0 + k) * 16.
+template <int MU, int NB>
 __device__ __forceinline__ void tc_issue_unit(uint32_t tmem, int acc0, uint32_t abuf, uint32_t bbuf, bool first) {
     constexpr int P = 32 / NB;
     const uint64_t da = tc_smem_desc_sw128(abuf);
@@ -138,10 +144,12 @@ __device__ __forceinline__ void tc_issue_unit(uint32_t tmem, int acc0, uint32_t 
     for (int k = 0; k < NB; ++k) {
         const uint32_t d = tmem + (uint32_t)((acc0 + k) * kTcN);
 #pragma unroll
-        for (int s = 0; s < P / 2; ++s) {
-            // K step s: 64-column block s/4, 32 bytes per step inside it (in 16-byte units)
-            const uint64_t a_off = (uint64_t)(((k * (P / 8) + s / 4) * (kTcRows / 8)) * 64 + (s % 4) * 2);
-            const uint64_t b_off = (uint64_t)(((k * (P / 8) + s / 4) * (kTcN / 8)) * 64 + (s % 4) * 2);
+        for (int s = 0; s < P * MU / 16; ++s) {
+            // K step s starts at chunk ck0 = (k*P*MU + 16 s)/8: atom ck0/8, then
+            // 16 bytes per chunk inside it (offsets in 16-byte units)
+            const int ck0 = (k * P * MU) / 8 + 2 * s;
+            const uint64_t a_off = (uint64_t)((ck0 >> 3) * (kTcRows / 8) * 64 + (ck0 & 7));
+            const uint64_t b_off = (uint64_t)((ck0 >> 3) * (kTcN / 8) * 64 + (ck0 & 7));
             asm volatile(
                 "{\n\t.reg .pred p;\n\t"
                 "setp.ne.b32 p, %4, 0;\n\t"
@@ -223,12 +231,27 @@ __device__ __forceinline__ uint2 ld_stream64(const void* p) {
 // Bytes 8*quarter .. 8*quarter+7 of row `slab*32 + lane` in unit u (zeros
 // past the last slab): half (quarter % 2) of the lane's (quarter / 2)-th
 // 128-bit word of the unit's chunk.
-template <int NB0, int NB1>
+__device__ __forceinline__ uint32_t ld_stream32(const void* p) {
+    uint32_t v;
+    asm volatile("ld.global.nc.L1::no_allocate.u32 %0, [%1];" : "=r"(v) : "l"(p));
+    return v;
+}
+
+// MU = 8: bytes 8*quarter .. +7 of row `slab*32 + lane` in unit u (half
+// quarter%2 of the lane's (quarter/2)-th 128-bit word of the unit's chunk);
+// MU = 4: word `quarter` of the lane's one 128-bit word.  Zeros past the last
+// slab.
+template <int MU, int NB0, int NB1>
 __device__ __forceinline__ void tc_load_words(const TcArgs& a, int u, int slab, int lane, int quarter, uint2& w) {
     const TcUnit t = tc_unit<NB0, NB1>(a, u);
-    w = slab < a.Ms ? ld_stream64(reinterpret_cast<const char*>(t.words + ((int64_t)slab * t.U + t.ul) * 64 +
-                                                                 (quarter >> 1) * 32 + lane) + 8 * (quarter & 1))
-                    : make_uint2(0, 0);
+    const uint4* chunk = t.words + ((int64_t)slab * t.U + t.ul) * (8 * MU);
+    if (slab >= a.Ms) {
+        w = make_uint2(0, 0);
+    } else if (MU == 8) {
+        w = ld_stream64(reinterpret_cast<const char*>(chunk + (quarter >> 1) * 32 + lane) + 8 * (quarter & 1));
+    } else {
+        w = make_uint2(ld_stream32(reinterpret_cast<const char*>(chunk + lane) + 4 * quarter), 0u);
+    }
 }
 
 // Writes the fp16 +-1 expansion of a quarter of one row's sign bytes (steps
@@ -237,20 +260,30 @@ __device__ __forceinline__ void tc_load_words(const TcArgs& a, int u, int slab, 
 // order).  At iteration it the lane takes the step whose chunk lands in
 // swizzled slot (it + L) mod 8, so the 8 rows of an atom store to 8 distinct
 // bank groups.
-template <int NB>
+template <int MU, int NB>
 __device__ __forceinline__ void tc_expand_quarter(uint32_t abuf, uint32_t lut, int row, int lane, int quarter,
                                                   const uint2& w) {
     constexpr int P = 32 / NB;
 #pragma unroll
     for (int it = 0; it < 8; ++it) {
-        const int qq = ((((it + lane) & 7) ^ (lane & 7)) - lane) & 7;
-        const int q = 8 * quarter + qq;
-        const uint32_t p = (qq < 4 ? w.x : w.y) >> (8 * (qq & 3));
-        const int k = ((q / P) + (lane / P)) % NB;
-        const int j = (lane + q) & (P - 1);
-        const uint2 lo = lds64(lut + ((p << 3) & 0x78u));
-        const uint2 hi = lds64(lut + ((p >> 1) & 0x78u));
-        sts128(abuf + sw128_chunk<NB>(k, j, row, kTcRows / 8), lo.x, lo.y, hi.x, hi.y);
+        if constexpr (MU == 8) {
+            const int qq = ((((it + lane) & 7) ^ (lane & 7)) - lane) & 7;
+            const int q = 8 * quarter + qq;
+            const uint32_t p = (qq < 4 ? w.x : w.y) >> (8 * (qq & 3));
+            const int k = ((q / P) + (lane / P)) % NB;
+            const int j = (lane + q) & (P - 1);
+            const uint2 lo = lds64(lut + ((p << 3) & 0x78u));
+            const uint2 hi = lds64(lut + ((p >> 1) & 0x78u));
+            sts128(abuf + sw128_block<MU, NB>(k, j, row, kTcRows / 8), lo.x, lo.y, hi.x, hi.y);
+        } else {
+            const int q = 8 * quarter + it;
+            const uint32_t p = w.x >> (4 * it);
+            const int k = ((q / P) + (lane / P)) % NB;
+            const int j = (lane + q) & (P - 1);
+            const uint2 v = lds64(lut + ((p << 3) & 0x78u));
+            asm volatile("st.shared.v2.b32 [%0], {%1,%2};" ::"r"(abuf + sw128_block<MU, NB>(k, j, row, kTcRows / 8)),
+                         "r"(v.x), "r"(v.y) : "memory");
+        }
     }
 }
 
@@ -266,14 +299,16 @@ struct TcProd {
     uint4 x;          // 8 fp16 activations of the batch row
 };
 
-template <int NB0, int NB1>
+template <int MU, int NB0, int NB1>
 __device__ __forceinline__ void tc_prod_load(const TcArgs& a, int u, int tid, TcProd& o) {
     const TcUnit t = tc_unit<NB0, NB1>(a, u);
     const int P = 32 / t.nb;
     const int b = tid & 15;
+    if ((tid >> 4) >= 4 * MU) return;   // the unit has 4*MU chunks of 8 columns
     {
-        const int kj = tid >> 4, k = kj / P, j = kj % P;
-        const int n0 = (t.ul * P + j) * 8;
+        // chunk tid/16 of the unit's K axis: base k, columns n0 .. n0+7 of the branch
+        const int kk0 = (tid >> 4) * 8, k = kk0 / (P * MU);
+        const int n0 = t.ul * P * MU + kk0 % (P * MU);
         if (!t.br && !t.gather && a.vec_x && n0 + 8 <= t.ncols) {
             o.c = __ldg(reinterpret_cast<const uint4*>(t.c + (int64_t)k * t.ncols + n0));
             o.x = b < a.B ? __ldg(reinterpret_cast<const uint4*>(a.x + (int64_t)b * a.N + n0))
@@ -306,11 +341,14 @@ __device__ __forceinline__ uint32_t mul_h2(uint32_t c, uint32_t x) {
     return *reinterpret_cast<const uint32_t*>(&hv);
 }
 
-template <int NB>
+template <int MU, int NB>
 __device__ __forceinline__ void tc_prod_store(const TcProd& o, int tid, uint32_t bbuf) {
     constexpr int P = 32 / NB;
-    const int b = tid & 15, kj = tid >> 4;
-    sts128(bbuf + sw128_chunk<NB>(kj / P, kj % P, b, kTcN / 8), mul_h2(o.c.x, o.x.x), mul_h2(o.c.y, o.x.y),
+    const int b = tid & 15, ck = tid >> 4;
+    if (ck >= 4 * MU) return;
+    // chunk ck holds 8 consecutive K of the unit: block (k, j) with (k*P + j)*MU = 8*ck
+    const int kj = ck * 8 / MU;
+    sts128(bbuf + sw128_block<MU, NB>(kj / P, kj % P, b, kTcN / 8), mul_h2(o.c.x, o.x.x), mul_h2(o.c.y, o.x.y),
            mul_h2(o.c.z, o.x.z), mul_h2(o.c.w, o.x.w));
 }
 
@@ -351,7 +389,7 @@ __device__ __forceinline__ TcItem tc_item(const TcArgs& a, int item, int U) {
     return it;
 }
 
-template <int NB0, int NB1>
+template <int MU, int NB0, int NB1>
 __global__ void __launch_bounds__(kTcThreads + 32, 1) fluxbin_tc_kernel(const TcArgs a) {
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const uint32_t sb = smem_base();
@@ -411,10 +449,10 @@ __global__ void __launch_bounds__(kTcThreads + 32, 1) fluxbin_tc_kernel(const Tc
                     const uint32_t bbuf = sb + kTcBOff + (uint32_t)bf * kTcBBytes;
                     if (NB1 > 0 && br1) {
                         constexpr int NB1E = NB1 > 0 ? NB1 : 1;
-                        tc_issue_unit<NB1E>(tmem, NB0, abuf, bbuf, first1);
+                        tc_issue_unit<MU, NB1E>(tmem, NB0, abuf, bbuf, first1);
                         first1 = false;
                     } else {
-                        tc_issue_unit<NB0>(tmem, 0, abuf, bbuf, first0);
+                        tc_issue_unit<MU, NB0>(tmem, 0, abuf, bbuf, first0);
                         first0 = false;
                     }
                     tc_commit(empty0 + 8u * bf);
@@ -439,20 +477,20 @@ __global__ void __launch_bounds__(kTcThreads + 32, 1) fluxbin_tc_kernel(const Tc
             uint2 wq[2];                         // this thread's 8 packed bytes of units u and u+1 (ring by parity)
             const bool early = (a.flags & kFlagEarlyWeights) != 0 || waited;
             if (early) {
-                if (u_begin < u_end) tc_load_words<NB0, NB1>(a, u_begin, slab, lane, quarter, wq[0]);
-                if (u_begin + 1 < u_end) tc_load_words<NB0, NB1>(a, u_begin + 1, slab, lane, quarter, wq[1]);
+                if (u_begin < u_end) tc_load_words<MU, NB0, NB1>(a, u_begin, slab, lane, quarter, wq[0]);
+                if (u_begin + 1 < u_end) tc_load_words<MU, NB0, NB1>(a, u_begin + 1, slab, lane, quarter, wq[1]);
             }
             if (!waited) {
                 asm volatile("griddepcontrol.wait;" ::: "memory");
                 waited = true;
             }
             if (!early) {
-                if (u_begin < u_end) tc_load_words<NB0, NB1>(a, u_begin, slab, lane, quarter, wq[0]);
-                if (u_begin + 1 < u_end) tc_load_words<NB0, NB1>(a, u_begin + 1, slab, lane, quarter, wq[1]);
+                if (u_begin < u_end) tc_load_words<MU, NB0, NB1>(a, u_begin, slab, lane, quarter, wq[0]);
+                if (u_begin + 1 < u_end) tc_load_words<MU, NB0, NB1>(a, u_begin + 1, slab, lane, quarter, wq[1]);
             }
             TcProd pq[2];                        // product operands of units u and u+1 (ring by parity)
-            if (u_begin < u_end) tc_prod_load<NB0, NB1>(a, u_begin, tid, pq[0]);
-            if (u_begin + 1 < u_end) tc_prod_load<NB0, NB1>(a, u_begin + 1, tid, pq[1]);
+            if (u_begin < u_end) tc_prod_load<MU, NB0, NB1>(a, u_begin, tid, pq[0]);
+            if (u_begin + 1 < u_end) tc_prod_load<MU, NB0, NB1>(a, u_begin + 1, tid, pq[1]);
             // per-row scales of this thread's row
             float rsc[2][4];
 #pragma unroll
@@ -476,20 +514,20 @@ __global__ void __launch_bounds__(kTcThreads + 32, 1) fluxbin_tc_kernel(const Tc
                 const TcProd pc = par ? pq[1] : pq[0];
                 if (u + 2 < u_end) {
                     if (par) {
-                        tc_load_words<NB0, NB1>(a, u + 2, slab, lane, quarter, wq[1]);
-                        tc_prod_load<NB0, NB1>(a, u + 2, tid, pq[1]);
+                        tc_load_words<MU, NB0, NB1>(a, u + 2, slab, lane, quarter, wq[1]);
+                        tc_prod_load<MU, NB0, NB1>(a, u + 2, tid, pq[1]);
                     } else {
-                        tc_load_words<NB0, NB1>(a, u + 2, slab, lane, quarter, wq[0]);
-                        tc_prod_load<NB0, NB1>(a, u + 2, tid, pq[0]);
+                        tc_load_words<MU, NB0, NB1>(a, u + 2, slab, lane, quarter, wq[0]);
+                        tc_prod_load<MU, NB0, NB1>(a, u + 2, tid, pq[0]);
                     }
                 }
                 if (NB1 > 0 && br1) {
                     constexpr int NB1E = NB1 > 0 ? NB1 : 1;
-                    tc_prod_store<NB1E>(pc, tid, bbuf);
-                    tc_expand_quarter<NB1E>(abuf, sb + kTcLutOff, row, lane, quarter, cur);
+                    tc_prod_store<MU, NB1E>(pc, tid, bbuf);
+                    tc_expand_quarter<MU, NB1E>(abuf, sb + kTcLutOff, row, lane, quarter, cur);
                 } else {
-                    tc_prod_store<NB0>(pc, tid, bbuf);
-                    tc_expand_quarter<NB0>(abuf, sb + kTcLutOff, row, lane, quarter, cur);
+                    tc_prod_store<MU, NB0>(pc, tid, bbuf);
+                    tc_expand_quarter<MU, NB0>(abuf, sb + kTcLutOff, row, lane, quarter, cur);
                 }
                 fence_async_smem();
                 tc_fence_before();

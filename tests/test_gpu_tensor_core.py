@@ -38,6 +38,10 @@ CASES = [
     (spec(33, 8192, 2, 2, 246, 8), 12),      # one ragged tile, units split over many items
     (spec(4096, 4096, 2, 1, 205, 8), 16),
     (spec(11008, 4096, 2, 1, 205, 8), 3),
+    (spec(300, 1024, 2, 2, 64, 4), 16),      # mu = 4
+    (spec(1000, 777, 1, 1, 100, 4), 8),
+    (spec(257, 2048, 4, 4, 33, 4), 16),
+    (spec(28672 // 8, 8192, 2, 2, 246, 4), 16),
 ]
 
 
@@ -52,7 +56,8 @@ def test_tc_parity_random(sp, B):
 
 def test_tc_exact_arithmetic_is_bit_exact():
     for i, (sp, B) in enumerate([(spec(2100, 777, 2, 1, 40, 8), 16), (spec(1030, 1500, 1, 2, 100, 8), 9),
-                                 (spec(200, 4096, 4, 1, 33, 8), 4)]):
+                                 (spec(200, 4096, 4, 1, 33, 8), 4), (spec(700, 1500, 2, 2, 90, 4), 16),
+                                 (spec(130, 600, 4, 4, 20, 4), 3)]):
         layer = synth.make_exact_layer(sp, [180, i])
         x = synth.make_exact_x(sp, B, [181, i])
         ref = oracle.linear(layer, x)
@@ -85,7 +90,8 @@ def test_tc_refuses_what_it_does_not_cover():
     x = torch.zeros((16, 512), dtype=torch.float16, device="cuda")
     y = torch.zeros((16, 256), dtype=torch.float32, device="cuda")
     for sp, status in ((spec(256, 512, 2, 0, 0, 8, G=128), -4),     # block-wise row scales
-                       (spec(256, 512, 2, 1, 40, 4), -4)):          # mu = 4
+                       (spec(256, 512, 2, 2, 256, 8, sal_scale_group=128), -4),  # block-wise salient scales
+                       (spec(256, 512, 2, 2, 64, 8, sal_scale_group=16), -4)):   # grouped salient scales
         d = fluxbin.DeviceLayer.from_host(synth.make_layer(sp, [194]))
         with pytest.raises(fluxbin.FluxbinError) as e:
             d.linear(x, y, TC, fluxbin.new_workspace(sp.M, 16))
