@@ -41,7 +41,7 @@
 //   tables  BT * 2^mu * 256: entry e of the tables of batch row b for unit
 //           parity h at b*2^mu*256 + e*256 + h*128 + bank*4 (consecutive units
 //           alternate halves: double buffering with one barrier per unit)
-//   vbuf    2 * BT * 32*mu floats: [parity][b][bank][t] activation products
+//   vbuf    2 * BT * 32*mu floats: [parity][b][t][bank] activation products
 //   red     BT * 528 floats: [b][source rank][row of this CTA's slice], the
 //           split-K partials the cluster's CTAs push to the slice owner
 //   scales  (grouped salient branch only) 2 * (32/gsv) * 512 fp16: the row
@@ -154,24 +154,27 @@ __device__ __forceinline__ T& smem_at(uint32_t byte_off) {
     return *reinterpret_cast<T*>(fb_smem + byte_off);
 }
 
-// Shared-memory access by 32-bit shared address (+ a constant byte offset).
+// Table entry at a byte offset from the start of the dynamic allocation (the
+// tables sit at offset 0).  An ordinary load through the shared array lets
+// the compiler fold the array's address into the load's immediate offset,
+// so a lookup costs one byte-permute and one load.
 template <int OFF>
-__device__ __forceinline__ float lds_f32(uint32_t addr) {
-    float v;
-    asm volatile("ld.shared.f32 %0, [%1+%2];" : "=f"(v) : "r"(addr), "n"(OFF));
+__device__ __forceinline__ float table_entry(uint32_t byte_off) {
+    return *reinterpret_cast<const float*>(fb_smem + OFF + byte_off);
+}
+
+// Shared-memory access by 32-bit shared address (+ a constant byte offset).
+__device__ __forceinline__ uint64_t lds_b64(uint32_t addr) {
+    uint64_t v;
+    asm volatile("ld.shared.b64 %0, [%1];" : "=l"(v) : "r"(addr));
     return v;
 }
-__device__ __forceinline__ float4 lds_f32x4(uint32_t addr) {
-    float4 v;
-    asm volatile("ld.shared.v4.f32 {%0,%1,%2,%3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(addr));
-    return v;
+template <int OFF>
+__device__ __forceinline__ void sts_b64_at(uint32_t addr, uint64_t v) {
+    asm volatile("st.shared.b64 [%0+%1], %2;" ::"r"(addr), "n"(OFF), "l"(v) : "memory");
 }
 __device__ __forceinline__ void sts_f32(uint32_t addr, float v) {
     asm volatile("st.shared.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
-}
-template <int OFF>
-__device__ __forceinline__ void sts_f32_at(uint32_t addr, float v) {
-    asm volatile("st.shared.f32 [%0+%1], %2;" ::"r"(addr), "n"(OFF), "f"(v) : "memory");
 }
 
 // Two fp32 values in one 64-bit register, added pairwise by one instruction.
@@ -183,6 +186,11 @@ __device__ __forceinline__ uint64_t pack_f32x2(float lo, float hi) {
 __device__ __forceinline__ uint64_t add_f32x2(uint64_t x, uint64_t y) {
     uint64_t z;
     asm("add.rn.f32x2 %0, %1, %2;" : "=l"(z) : "l"(x), "l"(y));
+    return z;
+}
+__device__ __forceinline__ uint64_t sub_f32x2(uint64_t x, uint64_t y) {
+    uint64_t z;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(z) : "l"(x), "l"(y));
     return z;
 }
 __device__ __forceinline__ float sum_f32x2(uint64_t x) {
@@ -262,7 +270,7 @@ __device__ __forceinline__ uint32_t word_of(const uint4& v, int i) {
 // pair (one paired fp32 add per two lookups) and folded into acc at the end.
 template <int MU, int NB, int HALF, int BT>
 __device__ __forceinline__ void lookup_unit(const uint4 (&w)[Geom<MU, BT>::kVecs], const Offsets<MU>& off,
-                                            uint32_t tbase, float (&acc)[BT][NB]) {
+                                            float (&acc)[BT][NB]) {
     constexpr int P = 32 / NB;
     constexpr int kStepsPerWord = 32 / MU;
     uint64_t pair[BT][NB];
@@ -273,13 +281,13 @@ __device__ __forceinline__ void lookup_unit(const uint4 (&w)[Geom<MU, BT>::kVecs
 #pragma unroll
     for (int q = 0; q < 32; q += 2) {
         const int wi0 = q / kStepsPerWord, wi1 = (q + 1) / kStepsPerWord;
-        const uint32_t a0 = tbase + off.addr(word_of(w[wi0 / 4], wi0 % 4), q);
-        const uint32_t a1 = tbase + off.addr(word_of(w[wi1 / 4], wi1 % 4), q + 1);
+        const uint32_t a0 = off.addr(word_of(w[wi0 / 4], wi0 % 4), q);
+        const uint32_t a1 = off.addr(word_of(w[wi1 / 4], wi1 % 4), q + 1);
         static_for<0, BT>([&](auto bc) {
             constexpr int b = decltype(bc)::value;
             constexpr int OFF = b * Geom<MU, BT>::kPairBytes + HALF * 128;
-            const float f0 = lds_f32<OFF>(a0);
-            const float f1 = lds_f32<OFF>(a1);
+            const float f0 = table_entry<OFF>(a0);
+            const float f1 = table_entry<OFF>(a1);
             pair[b][q / P] = add_f32x2(pair[b][q / P], pack_f32x2(f0, f1));
         });
     }
@@ -296,7 +304,7 @@ __device__ __forceinline__ void lookup_unit(const uint4 (&w)[Geom<MU, BT>::kVecs
 // One batch row (BT == 1).
 template <int MU, int NB, int GSV, int HALF>
 __device__ __forceinline__ void lookup_unit_grouped(const uint4 (&w)[kSlabsPerWarp][Geom<MU, 1>::kVecs],
-                                                    const Offsets<MU>& off, uint32_t tbase, uint32_t scale_row_off,
+                                                    const Offsets<MU>& off, uint32_t scale_row_off,
                                                     int lane, float (&tot)[kSlabsPerWarp][1]) {
     constexpr int kStepsPerWord = 32 / MU;
     constexpr int KG = 32 / GSV;
@@ -310,7 +318,7 @@ __device__ __forceinline__ void lookup_unit_grouped(const uint4 (&w)[kSlabsPerWa
             for (int e = 0; e < GSV; ++e) {
                 const int q = a * GSV + e;
                 const int wi = q / kStepsPerWord;
-                g += lds_f32<HALF * 128>(tbase + off.addr(word_of(w[rs][wi / 4], wi % 4), q));
+                g += table_entry<HALF * 128>(off.addr(word_of(w[rs][wi / 4], wi % 4), q));
             }
             const uint32_t kg = (uint32_t)((a + m) & (KG - 1));
             const float sc = __half2float(
@@ -320,7 +328,7 @@ __device__ __forceinline__ void lookup_unit_grouped(const uint4 (&w)[kSlabsPerWa
     }
 }
 
-// The activation-product slot a thread owns: bank c = s / mu, bit t = s % mu.
+// The activation-product slot a thread owns: bit t = s / 32, bank c = s % 32.
 struct SlotStatic {
     float c;   // column scale (0 for padding and out-of-range columns)
     int col;   // activation column (-1 for padding)
@@ -338,7 +346,7 @@ __device__ __forceinline__ SlotStatic slot_static(const KernelArgs& a, int u, in
     const int nb = br1 ? (NB1 > 0 ? NB1 : 1) : NB0;
     const int P = 32 / nb;
     const int ul = br1 ? u - a.br[0].units : u;
-    const int cb = s / MU, t = s % MU;
+    const int cb = s % 32, t = s / 32;
     const int k = cb / P, j = cb % P;
     const int64_t n = ((int64_t)ul * P + j) * MU + t;
     if (n < ncols) {
@@ -366,37 +374,48 @@ __device__ __forceinline__ void store_products(uint32_t sbase, int parity, int s
                 c * __half2float(xv[b]));
 }
 
-// Tables of one unit for BT batch rows.  Lane = bank = (base k, sub-vector j).
+// Tables of one unit for BT batch rows.  A thread builds the entries of one
+// block of 2^lo consecutive patterns for two adjacent banks (tables) at once:
+// both tables' values travel as one fp32 pair, so every Gray-code step is one
+// paired add and one 64-bit store.  Item (b, block, bank pair) = thread index
+// strided by the CTA size; the 16 bank pairs of a block are 16 consecutive
+// threads, so a half-warp stores 128 contiguous bytes.
 template <int MU, int HALF, int BT>
-__device__ __forceinline__ void build_unit(uint32_t sbase, int warp, int lane) {
+__device__ __forceinline__ void build_unit(uint32_t sbase, int tid) {
     using G = Geom<MU, BT>;
     constexpr int LO = G::kLo;
     constexpr int NBLK = G::kBlocks;
-    for (int z = warp; z < BT * NBLK; z += kWarps) {
-        const int bl = z / NBLK, hi = z % NBLK;
-        float v[MU];
-        const uint32_t va = sbase + G::kVbufOff + ((HALF * BT + bl) * G::kSlots + lane * MU) * 4;
+    constexpr int kItems = BT * NBLK * 16;
+    constexpr uint64_t kSign2 = 0x8000000080000000ull;
 #pragma unroll
-        for (int h = 0; h < MU / 4; ++h) {
-            const float4 f = lds_f32x4(va + 16 * h);
-            v[4 * h] = f.x;
-            v[4 * h + 1] = f.y;
-            v[4 * h + 2] = f.z;
-            v[4 * h + 3] = f.w;
+    for (int it0 = 0; it0 < kItems; it0 += kThreads) {
+        const int it = it0 + tid;
+        if (kItems % kThreads != 0 && it >= kItems) break;
+        const int bl = it / (NBLK * 16), hi = (it / 16) % NBLK, pj = it % 16;
+        const uint32_t va = sbase + G::kVbufOff + (uint32_t)(((HALF * BT + bl) * G::kSlots + 2 * pj) * 4);
+        // entry of pattern hi << lo: +v_t for the set high bits, -v_t otherwise
+        uint64_t T = 0;
+#pragma unroll
+        for (int t = LO; t < MU; ++t) {
+            const uint64_t flip = ((hi >> (t - LO)) & 1) ? 0ull : kSign2;
+            const uint64_t vt = lds_b64(va + t * 128) ^ flip;
+            T = t == LO ? vt : add_f32x2(T, vt);
         }
-        float T = 0.f;
+        uint64_t d[LO];
 #pragma unroll
-        for (int t = LO; t < MU; ++t) T += ((hi >> (t - LO)) & 1) ? v[t] : -v[t];
-#pragma unroll
-        for (int t = 0; t < LO; ++t) T -= v[t];
-        const uint32_t base = sbase + (uint32_t)(bl * G::kPairBytes + lane * 4) + (uint32_t)(hi << LO) * 256u;
-        sts_f32_at<HALF * 128>(base, T);
+        for (int t = 0; t < LO; ++t) {
+            const uint64_t vt = lds_b64(va + t * 128);
+            T = sub_f32x2(T, vt);
+            d[t] = add_f32x2(vt, vt);
+        }
+        const uint32_t base = sbase + (uint32_t)(bl * G::kPairBytes + pj * 8) + (uint32_t)(hi << LO) * 256u;
+        sts_b64_at<HALF * 128>(base, T);
         static_for<1, (1 << LO)>([&](auto ic) {
             constexpr int i = decltype(ic)::value;
             constexpr int t = lowest_bit(i);
             constexpr int g = i ^ (i >> 1);
-            T += ((g >> t) & 1) ? 2.f * v[t] : -2.f * v[t];
-            sts_f32_at<g * 256 + HALF * 128>(base, T);
+            T = ((g >> t) & 1) ? add_f32x2(T, d[t]) : sub_f32x2(T, d[t]);
+            sts_b64_at<g * 256 + HALF * 128>(base, T);
         });
     }
 }
@@ -525,7 +544,7 @@ __device__ __forceinline__ void unit_step(const KernelArgs& a, int u, int u_end,
     const BranchArgs& br = a.br[BR];
     constexpr int P = 32 / NB;
     constexpr bool kGrouped = BR == 1 && GS1 > 0;
-    build_unit<MU, HALF, BT>(sbase, warp, lane);
+    build_unit<MU, HALF, BT>(sbase, tid);
     if (tid < Geom<MU, BT>::kSlots && u + 1 < u_end) {
         store_products<MU, BT>(sbase, HALF ^ 1, tid, pp.c1, pp.x1);
         pp.c1 = pp.c2;
@@ -555,7 +574,7 @@ __device__ __forceinline__ void unit_step(const KernelArgs& a, int u, int u_end,
         const uint32_t scale_row_off = Geom<MU, 1>::kScaleOff +
             (uint32_t)((HALF * (32 / GS1)) * kRowsPerCta + (slab0 % kSlabsPerCta) * kLanes + lane) * 2u;
         (void)P;
-        lookup_unit_grouped<MU, NB, GS1, HALF>(cur, off, sbase, scale_row_off, lane, tot);
+        lookup_unit_grouped<MU, NB, GS1, HALF>(cur, off, scale_row_off, lane, tot);
     } else {
 #pragma unroll
         for (int rs = 0; rs < kSlabsPerWarp; ++rs) {
@@ -563,7 +582,7 @@ __device__ __forceinline__ void unit_step(const KernelArgs& a, int u, int u_end,
 #pragma unroll
             for (int h = 0; h < Geom<MU, BT>::kVecs; ++h) cur[h] = wb.w[HALF][rs][h];
             if (u + 2 < u_end) load_unit_slab<MU, BT>(a, u + 2, slab0 + rs, lane, wb.w[HALF][rs]);
-            lookup_unit<MU, NB, HALF, BT>(cur, off, sbase, acc[rs]);
+            lookup_unit<MU, NB, HALF, BT>(cur, off, acc[rs]);
         }
     }
     if (!kGrouped && br.rgroup > 0) {
