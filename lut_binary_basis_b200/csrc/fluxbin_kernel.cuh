@@ -329,14 +329,18 @@ __device__ __forceinline__ void lookup_unit_grouped(const uint4 (&w)[kSlabsPerWa
 }
 
 // The activation-product slot a thread owns: bit t = s / 32, bank c = s % 32.
-struct SlotStatic {
-    float c;   // column scale (0 for padding and out-of-range columns)
-    int col;   // activation column (-1 for padding)
+// Its layer data (column scale, activation column) are requested a unit
+// before they are needed and kept as loaded: nothing at the request waits for
+// the loads.  The column is checked and the scale converted when the slot is
+// consumed.
+struct SlotRaw {
+    __half c;  // column scale (0 for padding)
+    int col;   // activation column as the column map holds it (-1 for padding)
 };
 
 template <int MU, int NB0, int NB1>
-__device__ __forceinline__ SlotStatic slot_static(const KernelArgs& a, int u, int s) {
-    SlotStatic r{0.f, -1};
+__device__ __forceinline__ SlotRaw slot_raw(const KernelArgs& a, int u, int s) {
+    SlotRaw r{__float2half(0.f), -1};
     const bool br1 = NB1 > 0 && u >= a.br[0].units;
     // select fields one by one (a reference chosen at run time would force a
     // local copy of the kernel parameters)
@@ -350,13 +354,22 @@ __device__ __forceinline__ SlotStatic slot_static(const KernelArgs& a, int u, in
     const int k = cb / P, j = cb % P;
     const int64_t n = ((int64_t)ul * P + j) * MU + t;
     if (n < ncols) {
-        const int cc = gptr ? __ldg(gptr + n) : (int)n;
-        if (cc >= 0 && cc < a.N) {
-            r.c = __half2float(cptr[(int64_t)k * ncols + n]);
-            r.col = cc;
-        }
+        r.col = gptr ? __ldg(gptr + n) : (int)n;
+        r.c = cptr[(int64_t)k * ncols + n];
     }
     return r;
+}
+
+// A consumed slot: its fp32 column scale (0 for padding and out-of-range
+// columns) and its activation column (-1 for those).
+struct SlotStatic {
+    float c;
+    int col;
+};
+
+__device__ __forceinline__ SlotStatic resolve_slot(const KernelArgs& a, const SlotRaw& r) {
+    const bool ok = r.col >= 0 && r.col < a.N;
+    return SlotStatic{ok ? __half2float(r.c) : 0.f, ok ? r.col : -1};
 }
 
 template <int BT>
@@ -438,14 +451,13 @@ __device__ __forceinline__ void load_unit_slab(const KernelArgs& a, int u, int s
 }
 
 // Per-thread state of the activation-product pipeline: the next unit's
-// products (column scale and activations loaded) and the column of the unit
-// after it (layer data loaded).
+// products (column scale and activations loaded) and the layer data of the
+// unit after it (requested, not yet consumed).
 template <int BT>
 struct ProductPipe {
     float c1;
     __half x1[BT];
-    float c2;
-    int col2;
+    SlotRaw s2;
 };
 
 template <int MU, int BT>
@@ -547,13 +559,10 @@ __device__ __forceinline__ void unit_step(const KernelArgs& a, int u, int u_end,
     build_unit<MU, HALF, BT>(sbase, tid);
     if (tid < Geom<MU, BT>::kSlots && u + 1 < u_end) {
         store_products<MU, BT>(sbase, HALF ^ 1, tid, pp.c1, pp.x1);
-        pp.c1 = pp.c2;
-        slot_x<BT>(a, b0, pp.col2, pp.x1);
-        if (u + 3 < u_end) {
-            const SlotStatic st = slot_static<MU, NB0, NB1>(a, u + 3, tid);
-            pp.c2 = st.c;
-            pp.col2 = st.col;
-        }
+        const SlotStatic st = resolve_slot(a, pp.s2);
+        pp.c1 = st.c;
+        slot_x<BT>(a, b0, st.col, pp.x1);
+        if (u + 3 < u_end) pp.s2 = slot_raw<MU, NB0, NB1>(a, u + 3, tid);
     }
     if constexpr (GS1 > 0) cp_async_wait_all();  // this unit's staged salient scales
     __syncthreads();
@@ -675,7 +684,7 @@ __global__ void __launch_bounds__(kThreads, min_blocks<BT>()) fluxbin_lut_kernel
     WeightRegs<MU, BT> wb;
     ScaleRing sr;
     float sc0[kSlabsPerWarp][NB0], sc1[kSlabsPerWarp][NB1E];
-    SlotStatic st0{0.f, -1}, st1{0.f, -1}, st2{0.f, -1};
+    SlotRaw st0{__float2half(0.f), -1}, st1 = st0, st2 = st0;
     const bool slot_owner = tid < G::kSlots;
     const bool early = (a.flags & kFlagEarlyWeights) != 0;
     auto fetch_layer = [&]() {
@@ -691,9 +700,9 @@ __global__ void __launch_bounds__(kThreads, min_blocks<BT>()) fluxbin_lut_kernel
         fetch_row_scales<NB0>(a, a.br[0], slab0, lane, sc0);
         if constexpr (NB1 > 0) fetch_row_scales<NB1>(a, a.br[1], slab0, lane, sc1);
         if (slot_owner) {
-            if (u_begin < u_end) st0 = slot_static<MU, NB0, NB1>(a, u_begin, tid);
-            if (u_begin + 1 < u_end) st1 = slot_static<MU, NB0, NB1>(a, u_begin + 1, tid);
-            if (u_begin + 2 < u_end) st2 = slot_static<MU, NB0, NB1>(a, u_begin + 2, tid);
+            if (u_begin < u_end) st0 = slot_raw<MU, NB0, NB1>(a, u_begin, tid);
+            if (u_begin + 1 < u_end) st1 = slot_raw<MU, NB0, NB1>(a, u_begin + 1, tid);
+            if (u_begin + 2 < u_end) st2 = slot_raw<MU, NB0, NB1>(a, u_begin + 2, tid);
         }
     };
     if (early) fetch_layer();
@@ -704,18 +713,18 @@ __global__ void __launch_bounds__(kThreads, min_blocks<BT>()) fluxbin_lut_kernel
     ProductPipe<BT> pp;
     if (slot_owner) {
         __half x0[BT];
-        slot_x<BT>(a, b0, st0.col, x0);
-        slot_x<BT>(a, b0, st1.col, pp.x1);
-        if (u_begin < u_end) store_products<MU, BT>(sbase, 0, tid, st0.c, x0);
+        const SlotStatic s0 = resolve_slot(a, st0), s1 = resolve_slot(a, st1);
+        slot_x<BT>(a, b0, s0.col, x0);
+        slot_x<BT>(a, b0, s1.col, pp.x1);
+        if (u_begin < u_end) store_products<MU, BT>(sbase, 0, tid, s0.c, x0);
+        pp.c1 = s1.c;
     }
     if constexpr (GS1 > 0) {
         if (u_begin < u_end && u_begin >= U0) stage_group_scales<MU, NB1, GS1>(a, u_begin, rg, tid, 0);
         cp_async_wait_all();
     }
     if (slot_owner) {
-        pp.c1 = st1.c;
-        pp.c2 = st2.c;
-        pp.col2 = st2.col;
+        pp.s2 = st2;
     }
     __syncthreads();
 
