@@ -384,6 +384,8 @@ def run_ours(args, rank, local_rank, world):
             "cublas_bf16_dense_gemv": cub,
             "clocks": clocks,
         }
+        if cub and cub.get("us_per_call"):
+            cub["lut_speedup_vs_dense"] = cub["us_per_call"] / us_per_call
         if args.sweep:
             result["sweep"] = run_sweep(device, l2, args)
     if world > 1:
@@ -437,14 +439,14 @@ def cublas_reference(layer, spec, B, device, l2, args):
             "lut_speedup_vs_dense": None}
 
 
-def time_layer(spec, B, device, l2, wid, steps=50):
+def time_layer(spec, B, device, l2, wid, steps=50, path_flags=0):
     import torch
     from lut_binary_basis_b200 import fluxbin, synth
     layer = synth.make_layer(spec, synth.layer_key(wid, 0, 0))
     copies, xs, ys, R = build_pool(layer, spec, B, device, l2)
     del layer
     ws = fluxbin.new_workspace(spec.M, B, device)
-    flags = fluxbin.FLAG_EARLY_WEIGHTS
+    flags = fluxbin.FLAG_EARLY_WEIGHTS | path_flags
     stream = torch.cuda.Stream(device)
     with torch.cuda.stream(stream):
         for i in range(R):
@@ -494,7 +496,9 @@ def run_one_layer(args):
     wid, sp = find_layer(args.layer)
     props = torch.cuda.get_device_properties(device)
     l2 = getattr(props, "L2_cache_size", 126 * 2 ** 20) or 126 * 2 ** 20
-    return time_layer(sp, args.batch, device, l2, wid, steps=args.steps)
+    from lut_binary_basis_b200 import fluxbin
+    path = {"auto": 0, "lut": fluxbin.FLAG_PATH_LUT, "tc": fluxbin.FLAG_PATH_TC}[args.path]
+    return {**time_layer(sp, args.batch, device, l2, wid, steps=args.steps, path_flags=path), "path": args.path}
 
 
 def run_sweep(device, l2, args):
@@ -567,7 +571,7 @@ def run_stack(args):
     layers = build_stack(device, n_layers, workers)
     setup_s = time.time() - t0
     ws = fluxbin.new_workspace(max(sp.M for sp, *_ in layers), 1, device)
-    flags = fluxbin.FLAG_EARLY_WEIGHTS
+    flags = fluxbin.FLAG_EARLY_WEIGHTS | path_flags
     stream = torch.cuda.Stream(device)
 
     def step():
@@ -657,6 +661,8 @@ def main(argv=None):
     ap.add_argument("--layer", default=None,
                     help="time one named layer of the workloads instead (e.g. llama7b_gate_up_11008x4096)")
     ap.add_argument("--batch", type=int, default=1)
+    ap.add_argument("--path", choices=("auto", "lut", "tc"), default="auto",
+                    help="with --layer: force the LUT or the tensor-core path (default: the library's choice)")
     ap.add_argument("--stack", action="store_true",
                     help="time the 32-layer LLaMA-2-7B-shaped stack of 2.75-bit linears instead")
     ap.add_argument("--stack-layers", type=int, default=32)
