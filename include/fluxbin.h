@@ -147,8 +147,9 @@ typedef struct fluxbin_layer_desc {
  * LUT Tensor Core notes, Section 2.2, read LUT-based mixed-precision GEMM as a
  * GEMM with one low-bit operand).  It needs mu == 4 or 8, per-row scales
  * (row_scale_group == 0 and sal_scale_group == 0) and a workspace; it is taken
- * by default when B >= 8 and the layer qualifies, and may be forced either way
- * with the flags above.  Its products are rounded to fp16 before the
+ * by default for a qualifying layer when B >= 16 and M * N > 4096 * 4096, or
+ * when B >= 8 and M >= 16384 (where it measured faster on B200), and may be
+ * forced either way with the flags above.  Its products are rounded to fp16 before the
  * contraction (relative error below 2^-11 per product).
  */
 

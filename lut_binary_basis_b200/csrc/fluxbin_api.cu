@@ -23,8 +23,15 @@ KernelFn select_kernel_mu4(int nb0, int nb1, int bt, int gs1);
 using TcKernelFn = void (*)(TcArgs);
 TcKernelFn select_tc_kernel(int mu, int nb0, int nb1);
 
-// Smallest batch the automatic path choice sends to the tensor cores.
-constexpr int kTcMinBatch = 8;
+// Automatic path choice for a layer both paths can run.  Measured on B200
+// (µs per call, LUT / tensor cores): 4096x4096 B=8 17.6/35.7, B=16 31.0/38.1;
+// 4096x11008 B=8 40.4/60.4, B=16 76.3/65.0; 11008x4096 B=8 58.9/58.7,
+// B=16 112.5/63.0; 28672x8192 B=8 244/183, B=16 451/196; 8192x28672 (mu=4)
+// B=8 241/255, B=16 473/256.  The tensor cores win from batch 16 on layers
+// above 4096x4096 and from batch 8 on layers with at least 16384 rows.
+static bool prefer_tensor_cores(int64_t M, int64_t N, int B) {
+    return (B >= 16 && M * N > (int64_t)4096 * 4096) || (B >= 8 && M >= 16384);
+}
 
 namespace {
 
@@ -319,7 +326,8 @@ int run(int32_t M, int32_t N, int mu, const BranchIn& g, const BranchIn* s, cons
     const bool tc_fits = (mu == 8 || mu == 4) && g.rgroup == 0 && (!nb1 || s->rgroup == 0);
     if ((flags & kFlagPathTc) && !tc_fits) return FLUXBIN_ERR_UNSUPPORTED;
     if ((flags & kFlagPathTc) ||
-        (!(flags & kFlagPathLut) && tc_fits && B >= kTcMinBatch && ws && ws_bytes >= workspace_bytes_for(M, B)))
+        (!(flags & kFlagPathLut) && tc_fits && prefer_tensor_cores(M, N, B) && ws &&
+         ws_bytes >= workspace_bytes_for(M, B)))
         return run_tc(M, N, mu, g, s, nb1, d_x, B, d_y, flags & ~(kFlagPathLut | kFlagPathTc), ws, ws_bytes, stream);
     // salient row scales finer than a unit: grouped visit order, one batch row per CTA
     const int gs1 = (nb1 && s->rgroup > 0 && s->rgroup < unit_cols(nb1, mu)) ? s->rgroup / mu : 0;

@@ -347,12 +347,13 @@ __device__ __forceinline__ SlotRaw slot_raw(const KernelArgs& a, int u, int s) {
     const __half* cptr = br1 ? a.br[1].c : a.br[0].c;
     const int32_t* gptr = br1 ? a.br[1].gather : a.br[0].gather;
     const int ncols = br1 ? a.br[1].ncols : a.br[0].ncols;
-    const int nb = br1 ? (NB1 > 0 ? NB1 : 1) : NB0;
-    const int P = 32 / nb;
+    // sub-vectors per base and unit of each branch (compile-time divisors)
+    constexpr int P0 = 32 / NB0, P1 = NB1 > 0 ? 32 / NB1 : 32;
     const int ul = br1 ? u - a.br[0].units : u;
     const int cb = s % 32, t = s / 32;
-    const int k = cb / P, j = cb % P;
-    const int64_t n = ((int64_t)ul * P + j) * MU + t;
+    const int k = br1 ? cb / P1 : cb / P0;
+    const int j = br1 ? cb % P1 : cb % P0;
+    const int64_t n = (int64_t)ul * (br1 ? P1 * MU : P0 * MU) + j * MU + t;
     if (n < ncols) {
         r.col = gptr ? __ldg(gptr + n) : (int)n;
         r.c = cptr[(int64_t)k * ncols + n];

@@ -1,8 +1,9 @@
 """GPU parity of the tensor-core path (fluxbin_tc.cuh) against the fp64 oracle.
 
 The path is forced with FLUXBIN_FLAG_PATH_TC so that every batch size and
-shape below runs on it; the default choice sends B >= 8 there on its own (the
-full-size B = 8 and B = 16 cases of test_gpu_parity.py).  Same tolerance as the
+shape below runs on it; the default choice sends batches of 16 on layers above
+4096x4096, and batches of 8 on layers of at least 16384 rows, there on its own
+(the full-size 70B-shaped B = 16 cases of test_gpu_parity.py).  Same tolerance as the
 LUT path; cases with small-integer activations and power-of-two scales are
 exact (products exact in fp16, sums exact in fp32) and must match bit for bit.
 """
