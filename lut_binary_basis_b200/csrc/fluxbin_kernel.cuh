@@ -614,11 +614,9 @@ template <int MU, int BR, int NB, int BT, int NB0, int NB1, int GS1>
 __device__ __forceinline__ void run_branch(const KernelArgs& a, int u_lo, int u_hi, int u_end, int& v, int b0, int rg,
                                            int slab0, int warp, int lane, int tid, uint32_t sbase,
                                            ProductPipe<BT>& pp, WeightRegs<MU, BT>& wb, ScaleRing& sr,
-                                           float (&acc)[kSlabsPerWarp][BT][NB],
+                                           const Offsets<MU>& off, float (&acc)[kSlabsPerWarp][BT][NB],
                                            float (&tot)[kSlabsPerWarp][BT]) {
     if (u_lo >= u_hi) return;
-    Offsets<MU> off;
-    off.template load<NB, BR == 1 ? GS1 : 0>(lane);
     const int ubase = BR ? a.br[0].units : 0;
     for (int u = u_lo; u < u_hi; ++u, ++v) {
         if (v & 1)
@@ -630,10 +628,12 @@ __device__ __forceinline__ void run_branch(const KernelArgs& a, int u_lo, int u_
     }
 }
 
-// Per-row scales of the lane's rows for one branch: sc[rs][a] = r_{k(a)}[row].
+// Per-row scales of the lane's rows for one branch: sc[rs][a] = r_{k(a)}[row],
+// kept in fp16 as loaded (converted where they are applied, after the last
+// unit, so that nothing waits for these loads).
 template <int NB>
 __device__ __forceinline__ void fetch_row_scales(const KernelArgs& a, const BranchArgs& br, int slab0, int lane,
-                                                 float (&sc)[kSlabsPerWarp][NB]) {
+                                                 __half (&sc)[kSlabsPerWarp][NB]) {
     constexpr int P = 32 / NB;
 #pragma unroll
     for (int rs = 0; rs < kSlabsPerWarp; ++rs) {
@@ -641,7 +641,8 @@ __device__ __forceinline__ void fetch_row_scales(const KernelArgs& a, const Bran
 #pragma unroll
         for (int ai = 0; ai < NB; ++ai) {
             const int k = (ai + lane / P) % NB;
-            sc[rs][ai] = (i < a.M && br.rgroup == 0 && br.units > 0) ? __half2float(br.r[(int64_t)k * a.M + i]) : 0.f;
+            sc[rs][ai] = __float2half(0.f);
+            if (i < a.M && br.rgroup == 0 && br.units > 0) sc[rs][ai] = br.r[(int64_t)k * a.M + i];
         }
     }
 }
@@ -684,7 +685,11 @@ __global__ void __launch_bounds__(kThreads, min_blocks<BT>()) fluxbin_lut_kernel
 
     WeightRegs<MU, BT> wb;
     ScaleRing sr;
-    float sc0[kSlabsPerWarp][NB0], sc1[kSlabsPerWarp][NB1E];
+    __half sc0[kSlabsPerWarp][NB0], sc1[kSlabsPerWarp][NB1E];
+    // visit offsets of the first branch (a constant table): requested before
+    // the dependency wait
+    Offsets<MU> off0;
+    off0.template load<NB0, 0>(lane);
     SlotRaw st0{__float2half(0.f), -1}, st1 = st0, st2 = st0;
     const bool slot_owner = tid < G::kSlots;
     const bool early = (a.flags & kFlagEarlyWeights) != 0;
@@ -745,10 +750,15 @@ __global__ void __launch_bounds__(kThreads, min_blocks<BT>()) fluxbin_lut_kernel
 
     int v = 0;
     run_branch<MU, 0, NB0, BT, NB0, NB1, GS1>(a, u_begin, min(u_end, U0), u_end, v, b0, rg, slab0, warp, lane, tid,
-                                              sbase, pp, wb, sr, acc0, tot);
-    if constexpr (NB1 > 0)
-        run_branch<MU, 1, NB1, BT, NB0, NB1, GS1>(a, max(u_begin, U0), u_end, u_end, v, b0, rg, slab0, warp, lane, tid,
-                                                  sbase, pp, wb, sr, acc1, tot);
+                                              sbase, pp, wb, sr, off0, acc0, tot);
+    if constexpr (NB1 > 0) {
+        if (max(u_begin, U0) < u_end) {
+            Offsets<MU> off1;
+            off1.template load<NB1, GS1>(lane);
+            run_branch<MU, 1, NB1, BT, NB0, NB1, GS1>(a, max(u_begin, U0), u_end, u_end, v, b0, rg, slab0, warp, lane,
+                                                      tid, sbase, pp, wb, sr, off1, acc1, tot);
+        }
+    }
 
     // Row scales (per-row case; the block-wise case was applied per unit).
 #pragma unroll
@@ -756,10 +766,10 @@ __global__ void __launch_bounds__(kThreads, min_blocks<BT>()) fluxbin_lut_kernel
 #pragma unroll
         for (int b = 0; b < BT; ++b) {
 #pragma unroll
-            for (int q = 0; q < NB0; ++q) tot[rs][b] = fmaf(sc0[rs][q], acc0[rs][b][q], tot[rs][b]);
+            for (int q = 0; q < NB0; ++q) tot[rs][b] = fmaf(__half2float(sc0[rs][q]), acc0[rs][b][q], tot[rs][b]);
             if constexpr (NB1 > 0) {
 #pragma unroll
-                for (int q = 0; q < NB1; ++q) tot[rs][b] = fmaf(sc1[rs][q], acc1[rs][b][q], tot[rs][b]);
+                for (int q = 0; q < NB1; ++q) tot[rs][b] = fmaf(__half2float(sc1[rs][q]), acc1[rs][b][q], tot[rs][b]);
             }
         }
 
