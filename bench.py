@@ -571,7 +571,7 @@ def run_stack(args):
     layers = build_stack(device, n_layers, workers)
     setup_s = time.time() - t0
     ws = fluxbin.new_workspace(max(sp.M for sp, *_ in layers), 1, device)
-    flags = fluxbin.FLAG_EARLY_WEIGHTS | path_flags
+    flags = fluxbin.FLAG_EARLY_WEIGHTS
     stream = torch.cuda.Stream(device)
 
     def step():
