@@ -204,7 +204,10 @@ int fluxbin_pack(const fluxbin_layer_desc* desc, const int8_t* signs, const int8
  * arrival counter per row group and batch chunk.  Host only.
  * The workspace must be zero-filled once before its first use (for example
  * with cudaMemsetAsync); every call leaves it zero-filled again.  Calls that
- * may run concurrently on the GPU must not share a workspace.
+ * may run concurrently on the GPU must not share a workspace.  Given one, a
+ * call may split long rows wider than a thread-block cluster and add the
+ * partial sums through it (their order of summation then varies from call to
+ * call); split-K reductions inside a cluster sum in a fixed order.
  * Errors: INVALID_ARG (null output), BAD_SHAPE (M < 0 or B < 0).
  */
 int fluxbin_workspace_bytes(int32_t M, int32_t B, size_t* bytes);

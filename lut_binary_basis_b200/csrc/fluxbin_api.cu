@@ -1,6 +1,7 @@
 // C-ABI device entry points of libfluxbin: argument validation, kernel
 // selection, grid sizing and the launch.  Declarations and the full contract
 // are in include/fluxbin.h.
+#include <algorithm>
 #include <cuda_runtime.h>
 
 #include <cstdio>
@@ -165,7 +166,7 @@ struct Plan {
 // leaves most SMs idle (few rows, long rows) the units are split as widely
 // as the SMs allow and reduced through the workspace.
 Plan make_plan(KernelFn fn, int dev, int mu, int bt, int gs1, int64_t Ms, int64_t U, int n_bc,
-               const DeviceInfo& di, const FuncInfo& fi) {
+               const DeviceInfo& di, const FuncInfo& fi, bool have_ws) {
     Plan p;
     p.n_rg = (int)((Ms + kSlabsPerCta - 1) / kSlabsPerCta);
     const int64_t groups = (int64_t)p.n_rg * n_bc;
@@ -174,6 +175,23 @@ Plan make_plan(KernelFn fn, int dev, int mu, int bt, int gs1, int64_t Ms, int64_
     if (want > U) want = U;
     if (want > kMaxCluster) want = kMaxCluster;
     const size_t smem = table_smem_bytes(mu, bt) + red_smem_bytes(bt) + scale_smem_bytes(gs1);
+    // Long rows on few row groups: a split wider than a cluster, reduced
+    // through the workspace, shortens each CTA's chain of units by more than
+    // the workspace reduction costs once a cluster would leave every CTA at
+    // least two more units (B200, batch 1: 4096x11008 8.5 us with a 30-way
+    // workspace split against 10.6 us with 16-CTA clusters; 4096x4096 and
+    // 11008x4096, where clusters leave 2-3 units per CTA, are faster with
+    // clusters).  Up to 85% of the slots (the rest stays free for the next
+    // call's early CTAs), then as few CTAs as give the same units per CTA.
+    // Only with a workspace from the caller.
+    const int64_t ks_cap = std::min<int64_t>(U, (slots * 17) / (20 * groups));
+    const int64_t units_wide = ks_cap >= 1 ? (U + ks_cap - 1) / ks_cap : U;
+    const int64_t ks_wide = (U + units_wide - 1) / units_wide;
+    if (have_ws && want >= 1 && ks_wide > kMaxCluster && (U + want - 1) / want >= units_wide + 2) {
+        p.n_ks = (int)ks_wide;
+        p.cluster = false;
+        return p;
+    }
     for (int64_t ks = want; ks >= 2; --ks) {
         if (groups * ks * 2 < di.sm_count) break;  // too few CTAs: use the workspace instead
         if (max_active_clusters(fn, dev, (int)ks, smem) >= groups) {
@@ -363,7 +381,8 @@ int run(int32_t M, int32_t N, int mu, const BranchIn& g, const BranchIn* s, cons
         if (st != FLUXBIN_OK) return st;
         st = func_info(fn, dev, mu, bt, gs1, di, &fi);
         if (st != FLUXBIN_OK) return st;
-        plan = make_plan(fn, dev, mu, bt, gs1, a.Ms, U, n_bc, di, fi);
+        const bool have_ws = ws && ws_bytes >= workspace_bytes_for(M, B) && aligned(ws, 16);
+        plan = make_plan(fn, dev, mu, bt, gs1, a.Ms, U, n_bc, di, fi, have_ws);
     }
     a.x = reinterpret_cast<const __half*>(d_x);
     a.y = d_y;
