@@ -37,6 +37,11 @@ if ROOT not in sys.path:
 
 METRIC = "LUT GEMV µs/call & achieved HBM GB/s (frac of ~8 TB/s peak), batch 1–16"
 NOMINAL_HBM_GBS = 8000.0
+# Shared-memory lookup roofline for batches >= 2 (one 4-byte table load per
+# weight byte, base and batch row at mu = 8): 32 loads per clock per SM at the
+# B200's maximum SM clock.
+LDS_PER_CLK_PER_SM = 32
+SM_MAX_MHZ = 1965.0
 FALLBACK_HBM_GBS = 6650.0
 
 
@@ -472,8 +477,12 @@ def time_layer(spec, B, device, l2, wid, steps=50, path_flags=0):
     peak, _ = measured_peaks()
     del g, copies, xs, ys
     torch.cuda.empty_cache()
+    lk = lookups(spec, B) / (us * 1e-6)
+    lds_peak = torch.cuda.get_device_properties(device).multi_processor_count * LDS_PER_CLK_PER_SM * SM_MAX_MHZ * 1e6
     return {"layer": spec.name, "B": B, "mu": spec.mu, "us_per_call": us, "GB/s": gbs, "frac_measured": gbs / peak,
-            "frac_nominal": gbs / NOMINAL_HBM_GBS, "lookups_per_s": lookups(spec, B) / (us * 1e-6),
+            "frac_nominal": gbs / NOMINAL_HBM_GBS, "lookups_per_s": lk,
+            "lookup_roofline": {"achieved": lk, "peak": lds_peak, "unit": "lookups/s", "frac": lk / lds_peak,
+                                "peak_source": "SMs x 32 shared loads per clock x 1965 MHz"},
             "copies": R}
 
 
