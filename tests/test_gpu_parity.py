@@ -213,7 +213,7 @@ def sampled_rows(M, n=48, seed=0):
 FULL = [
     (synth.layer_7b_proj(), [1], 1),
     (synth.layers_7b_mlp()[0], [1, 8], 2),
-    (synth.layers_7b_mlp()[1], [2, 4], 2),
+    (synth.layers_7b_mlp()[1], [1, 2, 4], 2),   # B = 1: split wider than a cluster through the workspace
     (synth.layers_70b_mlp(8)[0], [1], 3),
     (synth.layers_70b_mlp(8)[1], [16], 3),
     (synth.layers_70b_mlp(4)[0], [16], 3),
@@ -240,3 +240,28 @@ def test_parity_full_size_sampled_rows(sp, batches, wid):
         assert np.all(np.isfinite(got))
         ref = oracle.linear(layer, x, rows=rows)
         assert_close(got[:, rows], ref, layer, x)
+
+
+def test_long_rows_with_and_without_workspace():
+    """A layer with long rows on few row groups (4096x11008 at batch 1) is
+    split wider than a cluster through the caller's workspace; without one it
+    runs on clusters.  Both match the oracle, and the workspace is left zero."""
+    sp = synth.layers_7b_mlp()[1]
+    layer = synth.make_layer(sp, synth.layer_key(2, 0, 0))
+    d = fluxbin.DeviceLayer.from_host(layer)
+    rows = sampled_rows(sp.M)
+    x = synth.make_x(sp, 1, synth.x_key(2, 0, 0, 1))
+    ref = oracle.linear(layer, x, rows=rows)
+    xd = torch.from_numpy(x).cuda()
+    outs = []
+    for ws in (fluxbin.new_workspace(sp.M, 1), None):
+        y = torch.full((1, sp.M), float("nan"), dtype=torch.float32, device="cuda")
+        d.linear(xd, y, fluxbin.FLAG_Y_FP32, ws)
+        torch.cuda.synchronize()
+        got = y.cpu().numpy().astype(np.float64)
+        assert_close(got[:, rows], ref, layer, x)
+        if ws is not None:
+            assert int(ws.abs().sum().item()) == 0
+        outs.append(got)
+    # different split-K sums of the same products: equal within fp32 rounding
+    assert np.allclose(outs[0], outs[1], rtol=1e-4, atol=1e-3 * np.abs(outs[1]).max())
