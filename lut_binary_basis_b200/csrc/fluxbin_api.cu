@@ -21,6 +21,7 @@ namespace fluxbin {
 using KernelFn = void (*)(KernelArgs);
 KernelFn select_kernel_mu8(int nb0, int nb1, int bt, int gs1);
 KernelFn select_kernel_mu4(int nb0, int nb1, int bt, int gs1);
+KernelFn select_kernel_mu8_3(int nb0, int nb1, int bt, int gs1);
 using TcKernelFn = void (*)(TcArgs);
 TcKernelFn select_tc_kernel(int mu, int nb0, int nb1);
 
@@ -352,6 +353,12 @@ int run(int32_t M, int32_t N, int mu, const BranchIn& g, const BranchIn* s, cons
     const int bt = gs1 ? 1 : batch_tile(mu, B);
     KernelFn fn = mu == 8 ? select_kernel_mu8(g.nb, nb1, bt, gs1) : select_kernel_mu4(g.nb, nb1, bt, gs1);
     if (!fn) return FLUXBIN_ERR_UNSUPPORTED;
+    // Large layers at batch 1: three CTAs per SM (B200: 28672x8192 27.3 ->
+    // 25.8 us, 8192x28672 32.7 -> 29.5 us; the 7B-sized layers are 5-30%
+    // slower that way, their splits get too fine).
+    if (mu == 8 && B == 1 && (int64_t)M * N >= ((int64_t)1 << 27)) {
+        if (KernelFn f3 = select_kernel_mu8_3(g.nb, nb1, bt, gs1)) fn = f3;
+    }
 
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return FLUXBIN_ERR_CUDA;

@@ -660,12 +660,14 @@ __device__ __forceinline__ void store_y(const KernelArgs& a, int b, int i, float
 
 // Up to two CTAs per SM when one batch row is resident (their table builds
 // then overlap each other's lookups); larger batch tiles run one CTA per SM
-// with up to 255 registers a thread.
+// with up to 255 registers a thread.  Large layers at batch 1 may run a
+// build with three CTAs per SM (MB = 3, 80 registers a thread, a few bytes
+// spilled) whose extra warps hide more of the lookup latency.
 template <int BT>
 constexpr int min_blocks() { return BT == 1 ? 2 : 1; }
 
-template <int MU, int NB0, int NB1, int BT, int GS1>
-__global__ void __launch_bounds__(kThreads, min_blocks<BT>()) fluxbin_lut_kernel(const KernelArgs a) {
+template <int MU, int NB0, int NB1, int BT, int GS1, int MB = min_blocks<BT>()>
+__global__ void __launch_bounds__(kThreads, MB) fluxbin_lut_kernel(const KernelArgs a) {
     using G = Geom<MU, BT>;
     constexpr int NB1E = NB1 > 0 ? NB1 : 1;
     const int tid = threadIdx.x, warp = tid / kLanes, lane = tid % kLanes;
