@@ -490,7 +490,8 @@ def time_layer(spec, B, device, l2, wid, steps=50, path_flags=0):
     return {"layer": spec.name, "B": B, "mu": spec.mu, "us_per_call": us, "GB/s": gbs, "frac_measured": gbs / peak,
             "frac_nominal": gbs / NOMINAL_HBM_GBS, "lookups_per_s": lk,
             "lookup_roofline": {"achieved": lk, "peak": lds_peak, "unit": "lookups/s", "frac": lk / lds_peak,
-                                "peak_source": "SMs x 32 shared loads per clock x 1965 MHz"},
+                                "peak_source": "SMs x 32 shared loads per clock x 1965 MHz",
+                                "applies_to": "the LUT path (the tensor-core path makes no table lookups)"},
             "copies": R}
 
 
