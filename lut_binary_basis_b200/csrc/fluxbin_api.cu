@@ -47,8 +47,13 @@ int cuda_fail(cudaError_t e) {
 }
 
 // Batch rows whose tables a CTA keeps resident (the rest go to other CTAs).
+// At mu = 8 one row per CTA: two CTAs per SM, each streaming the weights
+// for its own batch row (mostly from L2 after the first), beat one CTA per
+// SM holding two rows' tables (B200, B = 2 / 4: 11008x4096 12.7 -> 11.4 /
+// 21.4 -> 18.7 us, 4096x11008 17.5 -> 13.0 / 27.4 -> 19.7 us, 4096x4096
+// 8.8 -> 6.6 / 12.1 -> 9.4 us).
 int batch_tile(int mu, int B) {
-    if (mu == 8) return B <= 1 ? 1 : 2;
+    if (mu == 8) return 1;
     return B <= 1 ? 1 : (B <= 2 ? 2 : 4);
 }
 

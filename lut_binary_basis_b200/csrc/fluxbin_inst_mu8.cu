@@ -50,9 +50,9 @@ KernelFn select_kernel_mu8_3(int nb0, int nb1, int bt, int gs1) {
     return (bt == 1 && gs1 == 0) ? pick3(nb0, nb1) : nullptr;
 }
 
-// Tables of one batch row take 64 KiB (two 32 KiB halves).  gs1 > 0: the
-// salient branch has row scales per group of gs1 sub-vectors (one batch row
-// per CTA).
+// Tables of one batch row take 64 KiB (two 32 KiB halves); one batch row per
+// CTA.  gs1 > 0: the salient branch has row scales per group of gs1
+// sub-vectors.
 KernelFn select_kernel_mu8(int nb0, int nb1, int bt, int gs1) {
     if (gs1 > 0) {
         if (bt != 1) return nullptr;
@@ -62,7 +62,6 @@ KernelFn select_kernel_mu8(int nb0, int nb1, int bt, int gs1) {
         return nullptr;
     }
     if (bt == 1) return pick<1, 0>(nb0, nb1);
-    if (bt == 2) return pick<2, 0>(nb0, nb1);
     return nullptr;
 }
 
