@@ -358,12 +358,7 @@ int run(int32_t M, int32_t N, int mu, const BranchIn& g, const BranchIn* s, cons
     const int bt = gs1 ? 1 : batch_tile(mu, B);
     KernelFn fn = mu == 8 ? select_kernel_mu8(g.nb, nb1, bt, gs1) : select_kernel_mu4(g.nb, nb1, bt, gs1);
     if (!fn) return FLUXBIN_ERR_UNSUPPORTED;
-    // Large layers at batch 1: three CTAs per SM (B200: 28672x8192 27.3 ->
-    // 25.8 us, 8192x28672 32.7 -> 29.5 us; the 7B-sized layers are 5-30%
-    // slower that way, their splits get too fine).
-    if (mu == 8 && B == 1 && (int64_t)M * N >= ((int64_t)1 << 27)) {
-        if (KernelFn f3 = select_kernel_mu8_3(g.nb, nb1, bt, gs1)) fn = f3;
-    }
+
 
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return FLUXBIN_ERR_CUDA;
@@ -395,6 +390,26 @@ int run(int32_t M, int32_t N, int mu, const BranchIn& g, const BranchIn* s, cons
         if (st != FLUXBIN_OK) return st;
         const bool have_ws = ws && ws_bytes >= workspace_bytes_for(M, B) && aligned(ws, 16);
         plan = make_plan(fn, dev, mu, bt, gs1, a.Ms, U, n_bc, di, fi, have_ws);
+        // The build with three CTAs per SM (80 registers, a few bytes spilled)
+        // pays where its extra slots widen the split: large layers (B200,
+        // batch 1: 28672x8192 27.3 -> 25.8 us, 8192x28672 32.7 -> 29.5 us;
+        // batch 2 / 4: 54.7 -> 49.3 / 92.2 -> 84.9 us), and layers that two
+        // CTAs per SM would not split at all (11008x4096 at batch 8: 50.8 ->
+        // 37.3 us).  Otherwise it is slower (7B-sized layers at batch 1-4 by
+        // 5-30%; 28672x8192 at batch 4, same split, 104.7 -> 136.1 us).
+        if (mu == 8) {
+            KernelFn f3 = select_kernel_mu8_3(g.nb, nb1, bt, gs1);
+            FuncInfo fi3;
+            if (f3 && func_info(f3, dev, mu, bt, gs1, di, &fi3) == FLUXBIN_OK) {
+                const Plan p3 = make_plan(f3, dev, mu, bt, gs1, a.Ms, U, n_bc, di, fi3, have_ws);
+                const bool large = (int64_t)M * N >= ((int64_t)1 << 27);
+                if ((large && (B == 1 || p3.n_ks > plan.n_ks)) || (plan.n_ks == 1 && p3.n_ks >= 2)) {
+                    fn = f3;
+                    fi = fi3;
+                    plan = p3;
+                }
+            }
+        }
     }
     a.x = reinterpret_cast<const __half*>(d_x);
     a.y = d_y;
