@@ -1,19 +1,29 @@
 """Benchmark of the FluxBin LUT GEMV hot path on B200.
 
-Metric: LUT GEMV us/call and achieved HBM GB/s (fraction of the HBM peak).
-Workload (N = 1): the LLaMA-2-7B-shaped 4096 x 4096 projection, batch 1,
-2 global bases + 205 salient columns (5%) with 1 extra base, mu = 8,
-fp16 activations with 0.5% outlier channels, fp16 output.
+Metric: LUT GEMV us/call and achieved HBM GB/s (fraction of the HBM peak),
+batch 1-16.
 
-A step is one replay of a CUDA graph holding R fluxbin_linear calls over R
-distinct resident copies of the layer (packed signs, scales, column map and
-activations), R chosen so the copies total >= 3x the L2 size: every call
-streams its weights from HBM.  `value` is the algorithmic bytes of all calls
-(packed signs + fp16 scales + int32 column map + fp16 x + fp16 y) per second,
-summed over ranks.  Multi-GPU runs are independent replicas (weak scaling).
+Headline workload (N = 1): the 70B-shaped MLP up projection 28672 x 8192,
+batch 1, 2 global bases + 246 salient columns (3%) with 2 extra bases,
+mu = 8, fp16 activations N(0,1) with 0.5% outlier channels x20, fp16 output
+-- the largest single-layer configuration, on which the batch-1 LUT GEMV is
+expected to approach the HBM roofline.  A step is one replay of a CUDA graph
+holding R fluxbin_linear calls over R distinct resident copies of the layer
+(packed signs, scales, column map and activations), R chosen so the copies
+total >= 3x the L2 size: every call streams its weights from HBM.  `value` is
+the algorithmic bytes of all calls (packed signs + fp16 scales + int32
+column map + fp16 x + fp16 y) per second, summed over ranks.  Multi-GPU runs
+are independent replicas (weak scaling).
 
---impl reference times the fp64 CPU oracle (all host cores) on a bounded
-sample of rows of the same layer, in the same metric.
+The same JSON line carries, under "configs", every other configuration
+timed the same way (the 4096 x 4096 projection; the 7B MLP shapes at batch
+1, 2, 4, 8; the 70B MLP shapes at mu = 8 and 4, batch 1 and 16), each with
+its graph-pipelined and serialised time per call, and under "stack" the
+32-layer 2.75-bit LLaMA-2-7B-shaped stack of linears under one CUDA graph.
+
+--impl reference times the fp64 CPU oracle (all host cores) on the bounded
+sample of the headline layer that the cpu_baseline leg uses, in the same
+metric.
 """
 from __future__ import annotations
 
@@ -88,17 +98,17 @@ def kernel_source_hash() -> str:
 
 
 def profiled_traffic(workload: str):
-    """DRAM bytes per launch from the committed ncu summary of this workload,
-    if it was taken on the current kernel sources (else None)."""
-    p = os.path.join(ROOT, "profiles", f"fluxbin_lut_kernel_{workload}.txt")
-    if not os.path.exists(p):
-        return None
-    text = open(p).read()
-    m_hash = re.search(r"^kernel_source_hash:\s*(\S+)", text, re.M)
-    m_tr = re.search(r"^dram_bytes_per_launch:\s*([0-9.eE+]+)", text, re.M)
-    if not m_hash or not m_tr or m_hash.group(1) != kernel_source_hash():
-        return None
-    return float(m_tr.group(1))
+    """DRAM bytes per launch from the committed ncu summary of this workload
+    (profiles/<kernel>_<workload>.txt), if it was taken on the current kernel
+    sources (else None)."""
+    import glob
+    for p in sorted(glob.glob(os.path.join(ROOT, "profiles", f"*_{workload}.txt"))):
+        text = open(p).read()
+        m_hash = re.search(r"^kernel_source_hash:\s*(\S+)", text, re.M)
+        m_tr = re.search(r"^dram_bytes_per_launch:\s*([0-9.eE+]+)", text, re.M)
+        if m_hash and m_tr and m_hash.group(1) == kernel_source_hash():
+            return float(m_tr.group(1))
+    return None
 
 
 # ----------------------------------------------------------------------------
@@ -211,54 +221,235 @@ def whole_job_gbs(bytes_per_rank_per_step: float, steps: int, world: int, max_se
 # CPU oracle timing (baseline / reference arm)
 # ----------------------------------------------------------------------------
 
-def oracle_rate(spec, layer, x, rows_per_step: int, steps: int, warmup: int):
+def cpu_model() -> str:
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.lower().startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+CPU_SAMPLE_ROWS = 8192
+
+
+def _median_time(fn, reps: int) -> float:
+    ts = []
+    for _ in range(reps):
+        t0 = time.perf_counter()
+        fn()
+        ts.append(time.perf_counter() - t0)
+    return statistics.median(ts)
+
+
+def cpu_baseline(spec, layer, x, rows: int = CPU_SAMPLE_ROWS, reps: int = 5):
+    """The fp64 oracle on the host cores over a bounded sample (the first
+    `rows` output rows of the layer), four ways: single-threaded and on all
+    cores, each as the full call (rows of W rebuilt from signs and scales, then
+    W x) and as the GEMV alone on rows rebuilt beforehand.  Medians of `reps`
+    runs; per-call times and GB/s are scaled from the sample to the whole call
+    (the call's algorithmic bytes).  `value` is the all-core full call."""
     import oracle
-    rows = np.arange(min(rows_per_step, spec.M), dtype=np.int64)
-    for _ in range(warmup):
-        oracle.linear(layer, x, rows=rows)
-    t0 = time.perf_counter()
-    for _ in range(steps):
-        oracle.linear(layer, x, rows=rows)
-    dt = time.perf_counter() - t0
-    frac = rows.size / spec.M
-    bytes_per_step = frac * algorithmic_bytes(spec, x.shape[0])
-    return bytes_per_step * steps / dt / 1e9, dt, oracle.num_threads(), rows.size
-
-
-def cpu_baseline(spec, layer, x, budget_s: float = 12.0):
-    """The oracle on all host cores over a bounded sample: repeated full calls
-    on the first 512 rows (row rebuild in fp64 + dot product), ~budget_s seconds."""
-    rows = 512
-    gbs, dt, cores, nrows = oracle_rate(spec, layer, x, rows, 1, 1)
-    reps = max(1, int(budget_s / max(dt, 1e-3)))
-    gbs, dt, cores, nrows = oracle_rate(spec, layer, x, rows, reps, 0)
-    return {"value": gbs, "unit": "GB/s", "cores": cores, "kind": "oracle",
-            "sample": f"fp64 C oracle (W rows rebuilt from signs and scales, then W x) on rows 0..{nrows - 1} of "
-                      f"{spec.M}, {reps} repetitions, {dt:.1f} s; GB/s counts that fraction of the call's "
-                      f"algorithmic bytes",
-            "us_per_call": dt / reps * spec.M / nrows * 1e6}
+    oracle.build()
+    rr = np.arange(min(rows, spec.M), dtype=np.int64)
+    frac = rr.size / spec.M
+    per_call = algorithmic_bytes(spec, x.shape[0])
+    cores = os.cpu_count() or 1
+    out = {}
+    W = oracle.rebuild_rows(layer, rr)
+    for name, threads in (("single_thread", 1), ("all_cores", cores)):
+        oracle.set_num_threads(threads)
+        oracle.linear(layer, x, rows=rr[:256])   # warm-up
+        full = _median_time(lambda: oracle.linear(layer, x, rows=rr), reps)
+        gemv = _median_time(lambda: oracle.gemv_rows(W, x), reps)
+        out[name] = {"threads": threads, "full_call_us": full / frac * 1e6, "gemv_only_us": gemv / frac * 1e6,
+                     "full_call_GB/s": per_call / (full / frac) / 1e9, "gemv_only_GB/s": per_call / (gemv / frac) / 1e9}
+    oracle.set_num_threads(cores)
+    del W
+    return {"value": out["all_cores"]["full_call_GB/s"], "unit": "GB/s", "cores": cores, "kind": "oracle",
+            "cpu_model": cpu_model(),
+            "sample": f"fp64 C oracle on output rows 0..{rr.size - 1} of {spec.M} ({spec.name}, batch "
+                      f"{x.shape[0]}); median of {reps} runs each, single-threaded and on all {cores} cores, "
+                      f"full call (rows of W rebuilt, then W x) and GEMV alone on rows rebuilt beforehand; "
+                      f"times and GB/s scaled from the sample to the whole call",
+            "us_per_call": out["all_cores"]["full_call_us"], **out}
 
 
 # ----------------------------------------------------------------------------
 # GPU arm
 # ----------------------------------------------------------------------------
 
-def build_pool(layer, spec, B, device, l2_bytes):
+L2_BYTES = 126 * 2 ** 20   # B200 L2
+
+
+def rotation_copies(spec, B, l2_bytes=L2_BYTES) -> int:
+    """Distinct resident copies of a layer that total more than 3x the L2 size."""
+    return max(4, int(math.ceil(3 * l2_bytes / algorithmic_bytes(spec, B))))
+
+
+def build_pool(layer, spec, B, device, l2_bytes, wid=1):
+    """R distinct resident copies of the layer (and R inputs and outputs),
+    R chosen so that the copies total more than 3x the L2 size: every call of
+    a rotation streams its weights from HBM."""
     import torch
     from lut_binary_basis_b200 import fluxbin, synth
     base = fluxbin.DeviceLayer.from_host(layer, device)
-    per_copy = algorithmic_bytes(spec, B)
-    R = max(4, int(math.ceil(3 * l2_bytes / per_copy)))
-    copies, xs, ys = [], [], []
+    R = rotation_copies(spec, B, max(l2_bytes, L2_BYTES)) if l2_bytes > 2 * L2_BYTES else rotation_copies(spec, B)
+    copies, xs, ys = [base], [], []
     for i in range(R):
-        d = fluxbin.DeviceLayer(base.desc, base.words.clone(), base.r.clone(), base.c.clone(), base.swords.clone(),
-                                base.rs.clone(), base.cs.clone(), base.idx.clone())
-        copies.append(d)
-        x = synth.make_x(spec, B, synth.x_key(1, 0, i, B))
+        if i:
+            copies.append(fluxbin.DeviceLayer(base.desc, base.words.clone(), base.r.clone(), base.c.clone(),
+                                              base.swords.clone(), base.rs.clone(), base.cs.clone(),
+                                              base.idx.clone()))
+        x = synth.make_x(spec, B, synth.x_key(wid, 0, i, B))
         xs.append(torch.from_numpy(x).to(device))
         ys.append(torch.zeros((B, spec.M), dtype=torch.float16, device=device))
-    del base
     return copies, xs, ys, R
+
+
+def capture_rotation(copies, xs, ys, ws, flags, stream):
+    """One CUDA graph of the R calls of a rotation (after an eager run that also
+    sets the kernels' attributes outside the capture)."""
+    import torch
+    with torch.cuda.stream(stream):
+        for i in range(len(copies)):
+            copies[i].linear(xs[i], ys[i], flags, ws, stream)
+    stream.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for i in range(len(copies)):
+            copies[i].linear(xs[i], ys[i], flags, ws, stream)
+    stream.synchronize()
+    return g
+
+
+def time_graph(g, stream, steps: int, warmup: int = 3) -> float:
+    """Seconds per replay (CUDA events on the replay stream)."""
+    import torch
+    with torch.cuda.stream(stream):
+        for _ in range(warmup):
+            g.replay()
+    stream.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    with torch.cuda.stream(stream):
+        for _ in range(steps):
+            g.replay()
+    e1.record(stream)
+    stream.synchronize()
+    return e0.elapsed_time(e1) / 1e3 / steps
+
+
+def time_serialised(copies, xs, ys, ws, flags, stream, rounds: int = 3) -> float:
+    """Median seconds of one call on its own: every call bracketed by two CUDA
+    events, so it neither overlaps its predecessor nor is overlapped by its
+    successor.  The calls are queued behind a ~20 ms device sleep so that the
+    host's launch rate does not enter the timings."""
+    import torch
+    n = len(copies) * rounds
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+    with torch.cuda.stream(stream):
+        torch.cuda._sleep(40_000_000)
+        for k in range(n):
+            i = k % len(copies)
+            ev[k][0].record(stream)
+            copies[i].linear(xs[i], ys[i], flags, ws, stream)
+            ev[k][1].record(stream)
+    stream.synchronize()
+    return statistics.median(a.elapsed_time(b) for a, b in ev) / 1e3
+
+
+def lds_peak(device) -> float:
+    import torch
+    return torch.cuda.get_device_properties(device).multi_processor_count * LDS_PER_CLK_PER_SM * SM_MAX_MHZ * 1e6
+
+
+def layer_entry(spec, layer, B, device, l2, wid, steps=50, path_flags=0):
+    """µs per call of one layer at one batch size on the path the library
+    chooses (or the one forced): in a CUDA graph of R calls over R resident
+    copies (programmatic dependent launch lets each call start streaming its
+    weights while the previous one finishes), and serialised (median of single
+    calls).  GB/s and fractions count the call's algorithmic bytes."""
+    import torch
+    from lut_binary_basis_b200 import fluxbin
+    copies, xs, ys, R = build_pool(layer, spec, B, device, l2, wid)
+    ws = fluxbin.new_workspace(spec.M, B, device)
+    flags = fluxbin.FLAG_EARLY_WEIGHTS | path_flags
+    stream = torch.cuda.Stream(device)
+    g = capture_rotation(copies, xs, ys, ws, flags, stream)
+    us = time_graph(g, stream, steps) / R * 1e6
+    us_ser = time_serialised(copies, xs, ys, ws, flags, stream) * 1e6
+    del g, copies, xs, ys
+    torch.cuda.empty_cache()
+    per = algorithmic_bytes(spec, B)
+    peak, _ = measured_peaks()
+    gbs = per / (us * 1e-6) / 1e9
+    out = {"layer": spec.name, "M": spec.M, "N": spec.N, "Kb": spec.Kb, "Ks": spec.Ks, "n_sal": spec.n_sal,
+           "mu": spec.mu, "B": B, "us_per_call": us, "GB/s": gbs, "frac_measured": gbs / peak,
+           "frac_nominal": gbs / NOMINAL_HBM_GBS, "us_per_call_serialised": us_ser,
+           "frac_measured_serialised": per / (us_ser * 1e-6) / 1e9 / peak, "bytes_per_call": per, "copies": R}
+    if B >= 2:
+        lk = lookups(spec, B) / (us * 1e-6)
+        pk = lds_peak(device)
+        out["lookup_roofline"] = {"achieved": lk, "peak": pk, "unit": "lookups/s", "frac": lk / pk,
+                                  "peak_source": "SMs x 32 shared loads per clock x 1965 MHz",
+                                  "applies_to": "the LUT path (the tensor-core path makes no table lookups)"}
+    return out
+
+
+def config_layers():
+    """(workload id, layer spec, batches) of every benchmark configuration
+    other than the smallest (parity-only) one: the 4096x4096 projection, the
+    7B MLP shapes at batch 1-8, and the 70B MLP shapes at mu = 8 and 4,
+    batch 1 and 16."""
+    from lut_binary_basis_b200 import synth
+    out = [(1, synth.layer_7b_proj(), [1])]
+    out += [(2, sp, [1, 2, 4, 8]) for sp in synth.layers_7b_mlp()]
+    for mu in (8, 4):
+        out += [(3, sp, [1, 16]) for sp in synth.layers_70b_mlp(mu)]
+    return out
+
+
+def run_configs(device, l2, skip=None):
+    """Every configuration's layers at their batch sizes (the library's path
+    choice).  Layers of the same shape share one draw of signs and scales."""
+    import dataclasses
+    from lut_binary_basis_b200 import synth
+    out = {}
+    cache = {}
+    for wid, sp, batches in config_layers():
+        key = (wid, sp.M, sp.N)
+        if key not in cache:
+            cache.clear()
+            cache[key] = synth.make_layer(sp, synth.layer_key(wid, 0, 0))
+        layer = dataclasses.replace(cache[key], spec=sp)
+        for B in batches:
+            name = f"{sp.name}_b{B}"
+            if skip and name in skip:
+                out[name] = skip[name]
+                continue
+            out[name] = layer_entry(sp, layer, B, device, l2, wid)
+    return out
+
+
+HEADLINE_WID = 3
+
+
+def headline_spec():
+    from lut_binary_basis_b200 import synth
+    return synth.layers_70b_mlp(8)[0]
+
+
+def workload_config(spec, B, world):
+    """The `config` of the JSON line (identical in both arms)."""
+    R = rotation_copies(spec, B)
+    per_call = algorithmic_bytes(spec, B)
+    return {"workload": f"{spec.name}_b{B}", "M": spec.M, "N": spec.N, "Kb": spec.Kb, "Ks": spec.Ks,
+            "n_sal": spec.n_sal, "mu": spec.mu, "batch": B, "y": "fp16", "parallelism": f"replicas x{world}",
+            "calls_per_step": R,
+            "l2_policy": (f"inputs larger than L2: rotation over {R} distinct resident copies "
+                          f"({R * per_call / 2**20:.0f} MiB > 3x L2)")}
 
 
 def run_ours(args, rank, local_rank, world):
@@ -273,29 +464,21 @@ def run_ours(args, rank, local_rank, world):
         from datetime import timedelta
         dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=device)
 
-    spec = synth.layer_7b_proj()
+    spec = headline_spec()
     B = 1
-    layer = synth.make_layer(spec, synth.layer_key(1, 0, 0))
-    x_host = synth.make_x(spec, B, synth.x_key(1, 0, 0, B))
+    layer = synth.make_layer(spec, synth.layer_key(HEADLINE_WID, 0, 0))
+    x_host = synth.make_x(spec, B, synth.x_key(HEADLINE_WID, 0, 0, B))
     props = torch.cuda.get_device_properties(device)
     l2 = getattr(props, "L2_cache_size", 126 * 2 ** 20) or 126 * 2 ** 20
-    copies, xs, ys, R = build_pool(layer, spec, B, device, l2)
+    copies, xs, ys, R = build_pool(layer, spec, B, device, l2, HEADLINE_WID)
     ws = fluxbin.new_workspace(spec.M, B, device)
     flags = fluxbin.FLAG_EARLY_WEIGHTS  # fp16 y
 
     stream = torch.cuda.Stream(device)
+    g = capture_rotation(copies, xs, ys, ws, flags, stream)
     with torch.cuda.stream(stream):
-        for i in range(R):  # eager warm-up (also sets kernel attributes before capture)
-            copies[i].linear(xs[i], ys[i], flags, ws, stream)
-    stream.synchronize()
-    g = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g, stream=stream):
-        for i in range(R):
-            copies[i].linear(xs[i], ys[i], flags, ws, stream)
-    stream.synchronize()
-
-    for _ in range(args.warmup):
-        g.replay()
+        for _ in range(args.warmup):
+            g.replay()
     torch.cuda.synchronize(device)
 
     sampler = ClockSampler(gpu_id_for_smi(props)) if not args.no_clocks else None
@@ -327,6 +510,7 @@ def run_ours(args, rank, local_rank, world):
     us_per_call = max_secs / (args.steps * R) * 1e6
     achieved = per_call / (us_per_call * 1e-6) / 1e9
     peak, peak_kind = measured_peaks()
+    us_ser = time_serialised(copies, xs, ys, ws, flags, stream) * 1e6
 
     # end to end through the public API with host buffers: pinned x -> device,
     # the R calls, device y -> pinned host, every step (the step is captured
@@ -370,40 +554,51 @@ def run_ours(args, rank, local_rank, world):
 
     result = None
     if rank == 0:
-        cb = None
-        if not args.no_cpu:
-            cb = cpu_baseline(spec, layer, x_host)
-        cub = None if args.no_cublas else cublas_reference(layer, spec, B, device, l2, args)
         clocks = sampler.summary() if sampler else None
+        del g, g_e2e, copies, xs, ys, x_dev, y_dev
+        torch.cuda.empty_cache()
+        cb = None if args.no_cpu else cpu_baseline(spec, layer, x_host)
+        cub = None if args.no_cublas else cublas_reference(layer, spec, B, device, l2, args)
+        headline_name = f"{spec.name}_b{B}"
+        headline_entry = {"layer": spec.name, "M": spec.M, "N": spec.N, "Kb": spec.Kb, "Ks": spec.Ks,
+                          "n_sal": spec.n_sal, "mu": spec.mu, "B": B, "us_per_call": us_per_call,
+                          "GB/s": achieved, "frac_measured": achieved / peak,
+                          "frac_nominal": achieved / NOMINAL_HBM_GBS, "us_per_call_serialised": us_ser,
+                          "frac_measured_serialised": per_call / (us_ser * 1e-6) / 1e9 / peak,
+                          "bytes_per_call": per_call, "copies": R}
+        del layer
+        configs = None
+        if not args.headline_only:
+            configs = run_configs(device, l2, skip={headline_name: headline_entry})
+        stack = None if (args.headline_only or args.no_stack) else run_stack(args, device, summary=True)
         result = {
             "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": max_secs / args.steps * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic (seeded)",
-            "config": {"workload": "llama7b_proj_4096x4096_b1", "M": spec.M, "N": spec.N, "Kb": spec.Kb,
-                       "Ks": spec.Ks, "n_sal": spec.n_sal, "mu": spec.mu, "batch": B, "y": "fp16",
-                       "calls_per_step": R, "l2_policy": f"rotation over {R} distinct resident copies "
-                       f"({R * per_call / 2**20:.0f} MiB > 3x L2)", "parallelism": f"replicas x{world}"},
+            "config": workload_config(spec, B, world),
             "us_per_call": us_per_call,
+            "us_per_call_serialised": us_ser,
             "frac_of_nominal_8TBps": achieved / NOMINAL_HBM_GBS,
             "effective_tflops": 2.0 * spec.M * (spec.N + spec.n_sal) * B / (us_per_call * 1e-6) / 1e12,
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                         "frac": achieved / peak, "peak_source": peak_kind,
-                         "traffic": profiled_traffic("llama7b_proj_4096x4096_b1"),
-                         "bytes_per_launch": per_call},
+                         "frac": achieved / peak, "peak_source": f"{peak_kind} (HBM copy bandwidth)",
+                         "traffic": profiled_traffic(headline_name), "bytes_per_launch": per_call,
+                         "frac_serialised": per_call / (us_ser * 1e-6) / 1e9 / peak},
             "gpu_launches": R * args.steps,
             "e2e": {"value": e2e_value, "unit": "GB/s", "h2d_bytes_per_step": int(x_pin.numel() * 2),
                     "d2h_bytes_per_step": int(y_pin.numel() * 2), "steps": e2e_steps},
             "cpu_baseline": cb,
             "cublas_bf16_dense_gemv": cub,
             "clocks": clocks,
+            "configs": configs,
+            "stack": stack,
         }
         if cub and cub.get("us_per_call"):
             cub["lut_speedup_vs_dense"] = cub["us_per_call"] / us_per_call
-        if args.sweep:
-            result["sweep"] = run_sweep(device, l2, args)
+    else:
+        del g, g_e2e
     if world > 1:
         import torch.distributed as dist
-        del g, g_e2e
         dist.destroy_process_group()
     return result
 
@@ -415,6 +610,7 @@ def cublas_reference(layer, spec, B, device, l2, args):
     for k in range(spec.Kb):
         s = torch.from_numpy(layer.signs[k]).to(device).float()
         W += torch.from_numpy(layer.r[k]).to(device).float()[:, None] * s * torch.from_numpy(layer.c[k]).to(device).float()[None, :]
+        del s
     idx = torch.from_numpy(layer.sal_idx.astype(np.int64)).to(device)
     for k in range(layer.sal_signs.shape[0]):
         s = torch.from_numpy(layer.sal_signs[k]).to(device).float()
@@ -423,7 +619,7 @@ def cublas_reference(layer, spec, B, device, l2, args):
     del W
     per = Wb.numel() * 2
     R = max(4, int(math.ceil(3 * l2 / per)))
-    Ws = [Wb.clone() for _ in range(R)]
+    Ws = [Wb] + [Wb.clone() for _ in range(R - 1)]
     x = torch.randn((spec.N, B), dtype=torch.bfloat16, device=device)
     ys = [torch.empty((spec.M, B), dtype=torch.bfloat16, device=device) for _ in range(R)]
     stream = torch.cuda.Stream(device)
@@ -435,64 +631,13 @@ def cublas_reference(layer, spec, B, device, l2, args):
     with torch.cuda.graph(g, stream=stream):
         for i in range(R):
             torch.matmul(Ws[i], x, out=ys[i])
-    for _ in range(3):
-        g.replay()
-    torch.cuda.synchronize(device)
-    reps = 20
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    with torch.cuda.stream(stream):
-        for _ in range(reps):
-            g.replay()
-    e1.record(stream)
-    torch.cuda.synchronize(device)
-    us = e0.elapsed_time(e1) * 1e3 / (reps * R)
+    secs = time_graph(g, stream, 20)
+    us = secs * 1e6 / R
     gb = (per + 2 * B * (spec.M + spec.N)) / (us * 1e-6) / 1e9
-    return {"us_per_call": us, "GB/s_dense_bf16_bytes": gb, "copies": R,
-            "lut_speedup_vs_dense": None}
-
-
-def time_layer(spec, B, device, l2, wid, steps=50, path_flags=0):
-    import torch
-    from lut_binary_basis_b200 import fluxbin, synth
-    layer = synth.make_layer(spec, synth.layer_key(wid, 0, 0))
-    copies, xs, ys, R = build_pool(layer, spec, B, device, l2)
-    del layer
-    ws = fluxbin.new_workspace(spec.M, B, device)
-    flags = fluxbin.FLAG_EARLY_WEIGHTS | path_flags
-    stream = torch.cuda.Stream(device)
-    with torch.cuda.stream(stream):
-        for i in range(R):
-            copies[i].linear(xs[i], ys[i], flags, ws, stream)
-    stream.synchronize()
-    g = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g, stream=stream):
-        for i in range(R):
-            copies[i].linear(xs[i], ys[i], flags, ws, stream)
-    for _ in range(3):
-        g.replay()
-    torch.cuda.synchronize(device)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    with torch.cuda.stream(stream):
-        for _ in range(steps):
-            g.replay()
-    e1.record(stream)
-    torch.cuda.synchronize(device)
-    us = e0.elapsed_time(e1) * 1e3 / (steps * R)
-    per = algorithmic_bytes(spec, B)
-    gbs = per / (us * 1e-6) / 1e9
-    peak, _ = measured_peaks()
-    del g, copies, xs, ys
+    del g, Ws, ys, Wb
     torch.cuda.empty_cache()
-    lk = lookups(spec, B) / (us * 1e-6)
-    lds_peak = torch.cuda.get_device_properties(device).multi_processor_count * LDS_PER_CLK_PER_SM * SM_MAX_MHZ * 1e6
-    return {"layer": spec.name, "B": B, "mu": spec.mu, "us_per_call": us, "GB/s": gbs, "frac_measured": gbs / peak,
-            "frac_nominal": gbs / NOMINAL_HBM_GBS, "lookups_per_s": lk,
-            "lookup_roofline": {"achieved": lk, "peak": lds_peak, "unit": "lookups/s", "frac": lk / lds_peak,
-                                "peak_source": "SMs x 32 shared loads per clock x 1965 MHz",
-                                "applies_to": "the LUT path (the tensor-core path makes no table lookups)"},
-            "copies": R}
+    return {"us_per_call": us, "GB/s_dense_bf16_bytes": gb, "copies": R, "layer": spec.name, "B": B,
+            "lut_speedup_vs_dense": None}
 
 
 def find_layer(name):
@@ -508,26 +653,17 @@ def run_one_layer(args):
     """One layer of the workloads at one batch size (also the profiling driver)."""
     import torch
     import __graft_entry__
+    from lut_binary_basis_b200 import fluxbin, synth
     __graft_entry__.build()
     device = torch.device("cuda", 0)
     torch.cuda.set_device(device)
     wid, sp = find_layer(args.layer)
     props = torch.cuda.get_device_properties(device)
     l2 = getattr(props, "L2_cache_size", 126 * 2 ** 20) or 126 * 2 ** 20
-    from lut_binary_basis_b200 import fluxbin
     path = {"auto": 0, "lut": fluxbin.FLAG_PATH_LUT, "tc": fluxbin.FLAG_PATH_TC}[args.path]
-    return {**time_layer(sp, args.batch, device, l2, wid, steps=args.steps, path_flags=path), "path": args.path}
-
-
-def run_sweep(device, l2, args):
-    from lut_binary_basis_b200 import synth
-    out = []
-    for wid, specs, batches in ((2, synth.layers_7b_mlp(), [1, 2, 4, 8]),
-                                (3, synth.layers_70b_mlp(8) + synth.layers_70b_mlp(4), [1, 16])):
-        for sp in specs:
-            for B in batches:
-                out.append(time_layer(sp, B, device, l2, wid))
-    return out
+    layer = synth.make_layer(sp, synth.layer_key(wid, 0, 0))
+    return {**layer_entry(sp, layer, args.batch, device, l2, wid, steps=args.steps, path_flags=path),
+            "path": args.path}
 
 
 # ----------------------------------------------------------------------------
@@ -573,7 +709,7 @@ def stack_bits_per_weight(specs) -> float:
     return bits / w
 
 
-def run_stack(args):
+def run_stack(args, device=None, summary=False):
     """One decode step (batch 1) through all 224 linears, chained in order
     under one CUDA graph; a step's inputs are resident and the weights (2.2 GB)
     are far larger than L2."""
@@ -584,8 +720,9 @@ def run_stack(args):
     n_layers = args.stack_layers
     workers = max(1, min(8, (os.cpu_count() or 2) - 1))
     t0 = time.time()
-    device = torch.device("cuda", 0)
-    torch.cuda.set_device(device)
+    if device is None:
+        device = torch.device("cuda", 0)
+        torch.cuda.set_device(device)
     layers = build_stack(device, n_layers, workers)
     setup_s = time.time() - t0
     ws = fluxbin.new_workspace(max(sp.M for sp, *_ in layers), 1, device)
@@ -602,66 +739,72 @@ def run_stack(args):
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g, stream=stream):
         step()
-    for _ in range(args.warmup):
-        g.replay()
-    torch.cuda.synchronize(device)
-    props = torch.cuda.get_device_properties(device)
-    sampler = ClockSampler(gpu_id_for_smi(props)) if not args.no_clocks else None
-    if sampler:
+    steps = args.stack_steps if summary else args.steps
+    sampler = None
+    if not summary and not args.no_clocks:
+        sampler = ClockSampler(gpu_id_for_smi(torch.cuda.get_device_properties(device)))
         sampler.start()
         time.sleep(0.2)
         sampler.mark(True)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    with torch.cuda.stream(stream):
-        for _ in range(args.steps):
-            g.replay()
-    e1.record(stream)
-    torch.cuda.synchronize(device)
+    secs = time_graph(g, stream, steps, warmup=max(3, args.warmup if not summary else 3))
     if sampler:
         sampler.mark(False)
         sampler.stop()
-    secs = e0.elapsed_time(e1) / 1e3 / args.steps
     total = sum(algorithmic_bytes(sp, 1) for sp, *_ in layers)
+    n_linears = len(layers)
+    del g, layers
+    torch.cuda.empty_cache()
     peak, peak_kind = measured_peaks()
     gbs = total / secs / 1e9
     specs = synth.layers_7b_stack_linears()
-    return {"metric": "LLaMA-2-7B-shaped decoder stack, linears only: decode step time (batch 1)",
-            "value": secs * 1e6, "unit": "us/token", "higher_is_better": False, "n_gpus": 1,
-            "steps": args.steps, "warmup": args.warmup, "tokens_per_s": 1.0 / secs,
-            "dtype": "f32", "data": "synthetic (seeded)",
-            "config": {"workload": "llama7b_stack_32x7_275bit_b1", "layers": n_layers,
-                       "linears": len(layers), "bits_per_weight": stack_bits_per_weight(specs),
-                       "graph": "one CUDA graph, linears chained in order with programmatic dependent launch",
-                       "l2_policy": f"weights {total / 2**30:.2f} GiB per step > L2"},
-            "achieved_gbs": gbs, "roofline": {"bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s",
-                                              "frac": gbs / peak, "peak_source": peak_kind},
-            "gpu_launches": len(layers) * args.steps, "setup_s": setup_s,
-            "clocks": sampler.summary() if sampler else None}
+    res = {"metric": "LLaMA-2-7B-shaped decoder stack, linears only: decode step time (batch 1)",
+           "value": secs * 1e6, "unit": "us/token", "higher_is_better": False, "n_gpus": 1,
+           "steps": steps, "tokens_per_s": 1.0 / secs, "dtype": "f32", "data": "synthetic (seeded)",
+           "config": {"workload": "llama7b_stack_32x7_275bit_b1", "layers": n_layers,
+                      "linears": n_linears, "bits_per_weight": stack_bits_per_weight(specs),
+                      "graph": "one CUDA graph, linears chained in order with programmatic dependent launch",
+                      "l2_policy": f"weights {total / 2**30:.2f} GiB per step > L2"},
+           "achieved_gbs": gbs, "roofline": {"bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s",
+                                             "frac": gbs / peak, "peak_source": peak_kind},
+           "gpu_launches_per_step": n_linears, "setup_s": setup_s}
+    if not summary:
+        res.update({"warmup": args.warmup, "gpu_launches": n_linears * steps,
+                    "clocks": sampler.summary() if sampler else None})
+    return res
 
 
 def run_reference(args, rank, world):
-    """The oracle (CPU, all host cores) on a bounded sample of the same layer."""
+    """The oracle (CPU, all host cores): every step is one full call (rows of W
+    rebuilt from signs and scales, then W x) on the same bounded sample of the
+    benchmark's layer that the cpu_baseline leg times."""
     if rank != 0:
         return None
     from lut_binary_basis_b200 import synth
     import oracle
     oracle.build()
-    spec = synth.layer_7b_proj()
-    layer = synth.make_layer(spec, synth.layer_key(1, 0, 0))
-    x = synth.make_x(spec, 1, synth.x_key(1, 0, 0, 1))
-    rows_per_step = 32
-    gbs, dt, cores, nrows = oracle_rate(spec, layer, x, rows_per_step, args.steps, args.warmup)
-    us_per_call = dt / args.steps * spec.M / nrows * 1e6
-    sample = f"fp64 C oracle on rows 0..{nrows - 1} of {spec.M} per step (row rebuild + dot), {args.steps} steps"
+    spec = headline_spec()
+    layer = synth.make_layer(spec, synth.layer_key(HEADLINE_WID, 0, 0))
+    x = synth.make_x(spec, 1, synth.x_key(HEADLINE_WID, 0, 0, 1))
+    rr = np.arange(min(CPU_SAMPLE_ROWS, spec.M), dtype=np.int64)
+    frac = rr.size / spec.M
+    for _ in range(args.warmup):
+        oracle.linear(layer, x, rows=rr)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.linear(layer, x, rows=rr)
+    dt = time.perf_counter() - t0
+    per_call = algorithmic_bytes(spec, 1)
+    gbs = frac * per_call * args.steps / dt / 1e9 if dt > 0 else 0.0
+    cores = oracle.num_threads()
+    sample = (f"fp64 C oracle on all {cores} host cores ({cpu_model()}): output rows 0..{rr.size - 1} of "
+              f"{spec.M} per step (rows of W rebuilt, then W x), {args.steps} steps; GB/s counts that "
+              f"fraction of the call's algorithmic bytes")
+    cfg = workload_config(spec, 1, world)
     return {"impl": "reference", "metric": METRIC, "value": gbs, "unit": "GB/s", "n_gpus": world,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / max(args.steps, 1) * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic (seeded)",
-            "config": {"workload": "llama7b_proj_4096x4096_b1", "M": spec.M, "N": spec.N, "Kb": spec.Kb,
-                       "Ks": spec.Ks, "n_sal": spec.n_sal, "mu": spec.mu, "batch": 1,
-                       "parallelism": "host cores"},
-            "us_per_call": us_per_call,
+            "data": "synthetic (seeded)", "config": cfg,
+            "us_per_call": dt / max(args.steps, 1) / frac * 1e6,
             "cpu_baseline": {"kind": "oracle", "cores": cores, "sample": sample, "value": gbs, "unit": "GB/s"},
             "e2e": {"value": gbs, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
@@ -669,10 +812,13 @@ def run_reference(args, rank, world):
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--steps", type=int, default=500)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--sweep", action="store_true", help="also time the 7B MLP and 70B MLP layers at their batches")
+    ap.add_argument("--headline-only", action="store_true",
+                    help="time only the headline layer (no other configurations, no stack)")
+    ap.add_argument("--no-stack", action="store_true", help="skip the decoder-stack entry")
+    ap.add_argument("--stack-steps", type=int, default=20, help="graph replays timed for the stack entry")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-cublas", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")

@@ -136,6 +136,13 @@ typedef struct fluxbin_layer_desc {
 #define FLUXBIN_FLAG_PATH_LUT     8u  /* always use the LUT path */
 #define FLUXBIN_FLAG_PATH_TC      16u /* always use the tensor-core path (UNSUPPORTED when the layer
                                          does not qualify, WORKSPACE without a workspace) */
+#define FLUXBIN_FLAG_TEST_WAIT_TIMEOUT 32u /* test hook, only together with FLUXBIN_FLAG_PATH_TC: the
+                                         tensor-core kernel's preparing warps never report a buffer
+                                         ready and every wait gives up after a few polls, so the
+                                         give-up path runs: the outputs become NaN, bit 0 of
+                                         fluxbin_device_status is set, no MMA is issued, tensor
+                                         memory is released and the workspace is left zero-filled.
+                                         INVALID_ARG without FLUXBIN_FLAG_PATH_TC. */
 /*
  * Two execution paths compute the same layer.  The LUT path builds the 2^mu
  * signed partial sums of every activation sub-vector in shared memory and
@@ -161,10 +168,14 @@ const char* fluxbin_status_string(int status);
 const char* fluxbin_last_error(void);
 
 /*
- * Device-side status of the current device: bit 0 is set when a tensor-core
- * launch gave up waiting for its own tensor-core operations (never expected;
- * its outputs are then NaN).  Reads and clears the flags; synchronises with
- * the device.  Errors: INVALID_ARG (null output), CUDA.
+ * Device-side status of the current device.  Bit 0: a tensor-core launch gave
+ * up one of its bounded waits (never expected outside the test hook above;
+ * the outputs it owned are then NaN).  Bit 1: a tensor-core launch could not
+ * confirm that its matrix operations had finished and kept its tensor memory
+ * instead of releasing it under them (never expected).  The LUT path has no
+ * waits that can give up: its only cross-CTA wait is the hardware cluster
+ * barrier.  Reads and clears the flags; synchronises with the device.
+ * Errors: INVALID_ARG (null output), CUDA.
  */
 int fluxbin_device_status(uint32_t* out_flags);
 
@@ -273,8 +284,10 @@ int fluxbin_linear(const fluxbin_layer_desc* desc,
  *   - The first call on each device looks up the scratch address for that
  *     device (with the device current); make that first call before any
  *     stream capture begins.
- *   - Each call first clears, on `stream`, the part of the scratch that must
- *     start at zero (fluxbin_workspace_bytes(M, B) bytes), then launches.
+ *   - A call whose launch plan reduces its split-K partials through the
+ *     scratch first clears, on `stream`, the part that must start at zero
+ *     (fluxbin_workspace_bytes(M, B) bytes), then launches; a call whose plan
+ *     does not touch the scratch launches the layer alone.
  *   - Every call on a device shares the one scratch array: calls that may
  *     overlap on the GPU (different streams without ordering between them)
  *     race and give wrong results.  Order them on one stream.

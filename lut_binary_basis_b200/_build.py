@@ -20,7 +20,7 @@ LIB = os.path.join(PKG, "libfluxbin.so")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-Xcompiler", "-Wall",
               "--expt-relaxed-constexpr", "-I", os.path.join(ROOT, "include")] + ARCH
-CXX_FLAGS = ["-O2", "-std=c++17", "-fPIC", "-Wall", "-I", os.path.join(ROOT, "include")]
+CXX_FLAGS = ["-O3", "-std=c++17", "-fPIC", "-Wall", "-pthread", "-I", os.path.join(ROOT, "include")]
 
 CU_SOURCES = ["fluxbin_api.cu", "fluxbin_inst_mu8.cu", "fluxbin_inst_mu4.cu", "fluxbin_inst_tc.cu"]
 CXX_SOURCES = ["fluxbin_pack.cpp"]

@@ -243,7 +243,7 @@ int device_error_address(int dev, unsigned int** out) {
 // one CTA per SM; the unit ranges are split so that there are about four
 // items per SM.
 int run_tc(int32_t M, int32_t N, int mu, const BranchIn& g, const BranchIn* s, int nb1, const uint16_t* d_x, int32_t B,
-           void* d_y, uint32_t flags, void* ws, size_t ws_bytes, void* stream) {
+           void* d_y, uint32_t flags, void* ws, size_t ws_bytes, void* stream, int* uses_ws) {
     const size_t need = workspace_bytes_for(M, B);
     if (!ws || ws_bytes < need) return FLUXBIN_ERR_WORKSPACE;
     if (!aligned(ws, 16)) return FLUXBIN_ERR_MISALIGNED;
@@ -304,7 +304,13 @@ int run_tc(int32_t M, int32_t N, int mu, const BranchIn& g, const BranchIn* s, i
     if (ks < 1) ks = 1;
     a.n_ks = (int32_t)ks;
     a.n_items = a.n_rt * a.n_ks;
-    a.flags = flags;
+    if (uses_ws) {  // plan query only
+        *uses_ws = a.n_ks > 1 ? 1 : 0;
+        return FLUXBIN_OK;
+    }
+    a.test_stall = (flags & kFlagTestWaitTimeout) ? 1 : 0;
+    a.spin_limit = a.test_stall ? kTcTestSpinLimit : kTcSpinLimit;
+    a.flags = flags & ~kFlagTestWaitTimeout;
     const size_t acc = (((size_t)B * a.Mp * sizeof(float)) + 255) & ~(size_t)255;
     a.ws_acc = static_cast<float*>(ws);
     a.ws_cnt = reinterpret_cast<unsigned int*>(static_cast<char*>(ws) + acc);
@@ -326,11 +332,17 @@ int run_tc(int32_t M, int32_t N, int mu, const BranchIn& g, const BranchIn* s, i
     return FLUXBIN_OK;
 }
 
+// Validates the arguments, chooses the path and the launch plan and launches
+// the layer.  With `uses_ws` non-null nothing is launched: it reports whether
+// the chosen plan reduces through the workspace.
 int run(int32_t M, int32_t N, int mu, const BranchIn& g, const BranchIn* s, const uint16_t* d_x, int32_t B,
-        void* d_y, uint32_t flags, void* ws, size_t ws_bytes, void* stream) {
-    if (flags & ~(kFlagAccumulate | kFlagYFp32 | kFlagEarlyWeights | kFlagPathLut | kFlagPathTc))
+        void* d_y, uint32_t flags, void* ws, size_t ws_bytes, void* stream, int* uses_ws = nullptr) {
+    if (flags & ~(kFlagAccumulate | kFlagYFp32 | kFlagEarlyWeights | kFlagPathLut | kFlagPathTc |
+                  kFlagTestWaitTimeout))
         return FLUXBIN_ERR_INVALID_ARG;
     if ((flags & kFlagPathLut) && (flags & kFlagPathTc)) return FLUXBIN_ERR_INVALID_ARG;
+    if ((flags & kFlagTestWaitTimeout) && !(flags & kFlagPathTc)) return FLUXBIN_ERR_INVALID_ARG;
+    if (uses_ws) *uses_ws = 0;
     if (B < 0 || B > kMaxBatch) return B < 0 ? FLUXBIN_ERR_BAD_SHAPE : FLUXBIN_ERR_UNSUPPORTED;
     if (M == 0 || B == 0) return FLUXBIN_OK;
     if (!d_y || (N > 0 && !d_x)) return FLUXBIN_ERR_INVALID_ARG;
@@ -352,7 +364,8 @@ int run(int32_t M, int32_t N, int mu, const BranchIn& g, const BranchIn* s, cons
     if ((flags & kFlagPathTc) ||
         (!(flags & kFlagPathLut) && tc_fits && prefer_tensor_cores(M, N, B) && ws &&
          ws_bytes >= workspace_bytes_for(M, B)))
-        return run_tc(M, N, mu, g, s, nb1, d_x, B, d_y, flags & ~(kFlagPathLut | kFlagPathTc), ws, ws_bytes, stream);
+        return run_tc(M, N, mu, g, s, nb1, d_x, B, d_y, flags & ~(kFlagPathLut | kFlagPathTc), ws, ws_bytes, stream,
+                      uses_ws);
     // salient row scales finer than a unit: grouped visit order, one batch row per CTA
     const int gs1 = (nb1 && s->rgroup > 0 && s->rgroup < unit_cols(nb1, mu)) ? s->rgroup / mu : 0;
     const int bt = gs1 ? 1 : batch_tile(mu, B);
@@ -422,6 +435,10 @@ int run(int32_t M, int32_t N, int mu, const BranchIn& g, const BranchIn* s, cons
     a.n_ks = plan.n_ks;
     a.cluster = plan.cluster ? 1 : 0;
     a.flags = flags;
+    if (uses_ws) {  // plan query only
+        *uses_ws = (a.n_ks > 1 && !plan.cluster) ? 1 : 0;
+        return FLUXBIN_OK;
+    }
     if (a.n_ks > 1 && !plan.cluster) {
         const size_t need = workspace_bytes_for(M, B);
         if (!ws || ws_bytes < need) return FLUXBIN_ERR_WORKSPACE;
@@ -454,6 +471,21 @@ int run(int32_t M, int32_t N, int mu, const BranchIn& g, const BranchIn* s, cons
 }
 
 }  // namespace
+
+int linear_impl(const fluxbin_layer_desc* desc, const uint32_t* d_words, const uint16_t* d_r, const uint16_t* d_c,
+                const uint32_t* d_swords, const uint16_t* d_rs, const uint16_t* d_cs, const int32_t* d_idx,
+                const uint16_t* d_x, int32_t B, void* d_y, uint32_t flags, void* d_workspace,
+                size_t workspace_bytes, void* stream, int* uses_ws) {
+    const int st = validate_desc(desc);
+    if (st != FLUXBIN_OK) return st;
+    const fluxbin_layer_desc& d = *desc;
+    BranchIn g{d_words, d_r, d_c, nullptr, d.N, d.Kb, d.row_scale_group};
+    BranchIn s{d_swords, d_rs, d_cs, d_idx, has_salient(d) ? d.n_sal : 0, d.Ks ? d.Ks : 1, d.sal_scale_group};
+    if (has_salient(d) && !d_idx) return FLUXBIN_ERR_INVALID_ARG;
+    return run(d.M, d.N, d.mu, g, has_salient(d) ? &s : nullptr, d_x, B, d_y, flags, d_workspace,
+               workspace_bytes, stream, uses_ws);
+}
+
 }  // namespace fluxbin
 
 using namespace fluxbin;
@@ -496,14 +528,8 @@ int fluxbin_linear(const fluxbin_layer_desc* desc, const uint32_t* d_words, cons
                    const uint16_t* d_c, const uint32_t* d_swords, const uint16_t* d_rs, const uint16_t* d_cs,
                    const int32_t* d_idx, const uint16_t* d_x, int32_t B, void* d_y, uint32_t flags,
                    void* d_workspace, size_t workspace_bytes, void* stream) {
-    const int st = validate_desc(desc);
-    if (st != FLUXBIN_OK) return st;
-    const fluxbin_layer_desc& d = *desc;
-    BranchIn g{d_words, d_r, d_c, nullptr, d.N, d.Kb, d.row_scale_group};
-    BranchIn s{d_swords, d_rs, d_cs, d_idx, has_salient(d) ? d.n_sal : 0, d.Ks ? d.Ks : 1, d.sal_scale_group};
-    if (has_salient(d) && !d_idx) return FLUXBIN_ERR_INVALID_ARG;
-    return run(d.M, d.N, d.mu, g, has_salient(d) ? &s : nullptr, d_x, B, d_y, flags, d_workspace,
-               workspace_bytes, stream);
+    return linear_impl(desc, d_words, d_r, d_c, d_swords, d_rs, d_cs, d_idx, d_x, B, d_y, flags, d_workspace,
+                       workspace_bytes, stream, nullptr);
 }
 
 }  // extern "C"
@@ -561,11 +587,19 @@ extern "C" int fluxbin_linear_static_scratch(const fluxbin_layer_desc* desc, con
     void* scratch = nullptr;
     const int sa = static_scratch_address(&scratch);
     if (sa != FLUXBIN_OK) return sa;
-    // the previous call on this device may have left anything there
-    if (cudaMemsetAsync(scratch, 0, need, static_cast<cudaStream_t>(stream)) != cudaSuccess) {
+    // Plans that reduce inside a cluster or not at all never touch the
+    // scratch: those calls launch the layer alone (and keep their overlap with
+    // the previous kernel on the stream).  A plan that reduces through the
+    // scratch first clears the part it uses, since the previous call on this
+    // device may have left anything there.
+    int uses = 0;
+    int st2 = linear_impl(desc, d_words, d_r, d_c, d_swords, d_rs, d_cs, d_idx, d_x, B, d_y, flags, scratch,
+                          (size_t)FLUXBIN_STATIC_SCRATCH_BYTES, stream, &uses);
+    if (st2 != FLUXBIN_OK) return st2;
+    if (uses && cudaMemsetAsync(scratch, 0, need, static_cast<cudaStream_t>(stream)) != cudaSuccess) {
         (void)cudaGetLastError();
         return FLUXBIN_ERR_CUDA;
     }
-    return fluxbin_linear(desc, d_words, d_r, d_c, d_swords, d_rs, d_cs, d_idx, d_x, B, d_y, flags, scratch,
-                          (size_t)FLUXBIN_STATIC_SCRATCH_BYTES, stream);
+    return linear_impl(desc, d_words, d_r, d_c, d_swords, d_rs, d_cs, d_idx, d_x, B, d_y, flags, scratch,
+                       (size_t)FLUXBIN_STATIC_SCRATCH_BYTES, stream, nullptr);
 }

@@ -87,6 +87,7 @@ constexpr uint32_t kFlagYFp32 = 2u;
 constexpr uint32_t kFlagEarlyWeights = 4u;
 constexpr uint32_t kFlagPathLut = 8u;
 constexpr uint32_t kFlagPathTc = 16u;
+constexpr uint32_t kFlagTestWaitTimeout = 32u;
 
 template <int MU, int BT>
 struct Geom {

@@ -36,7 +36,13 @@
 //        8-byte entry per bank pair, so 32 lanes never conflict)
 //   bar  per buffer a "full" mbarrier (the 16 worker warps have prepared a
 //        unit) and an "empty" one (its MMAs have finished), then the
-//        tensor-memory address
+//        tensor-memory address and the issuer's drain flag
+//
+// Every mbarrier wait is bounded (spin_limit polls).  A wait that gives up
+// sets bit 0 of the device error word and the affected outputs become NaN;
+// the issuing thread then still waits (with the full limit) for the last
+// commit it made on each buffer, and the tensor memory is freed only once
+// those MMAs are known to have finished (bit 1 of the error word when not).
 #pragma once
 
 #include <cuda_fp16.h>
@@ -58,6 +64,7 @@ constexpr int kTcLutOff = kTcBOff + 2 * kTcBBytes;   // 16 x 8 B: fp16 +-1 of th
 constexpr int kTcBarOff = kTcLutOff + 128;
 constexpr int kTcSmemBytes = kTcBarOff + 48;
 constexpr uint32_t kTcSpinLimit = 1u << 26;   // mbarrier polls before a wait is declared failed
+constexpr uint32_t kTcTestSpinLimit = 64u;    // the same under the wait-timeout test hook
 
 struct TcArgs {
     BranchArgs br[2];       // 0: global, 1: salient (units == 0 when absent); per-row scales only
@@ -72,8 +79,10 @@ struct TcArgs {
     uint32_t flags;
     float* ws_acc;          // [B][Mp], zero between calls
     unsigned int* ws_cnt;   // [n_rt], zero between calls
-    unsigned int* err;      // set non-zero when a wait gives up (never expected)
+    unsigned int* err;      // bit 0: a wait gave up; bit 1: tensor memory kept (MMAs not drained)
     int32_t vec_x;          // 1: x rows and the global column scales allow 16-byte loads (N % 8 == 0, aligned)
+    uint32_t spin_limit;    // mbarrier polls before a wait gives up
+    int32_t test_stall;     // test hook: the workers never signal a buffer full
 };
 
 // ---------------------------------------------------------------------------
@@ -86,8 +95,8 @@ __device__ __forceinline__ void tc_mbar_init(uint32_t bar, uint32_t count) {
 
 // Polls the mbarrier until the phase with the given parity has completed;
 // false when the poll limit is reached.
-__device__ __forceinline__ bool tc_mbar_wait(uint32_t bar, uint32_t parity) {
-    for (uint32_t it = 0; it < kTcSpinLimit; ++it) {
+__device__ __forceinline__ bool tc_mbar_wait(uint32_t bar, uint32_t parity, uint32_t limit) {
+    for (uint32_t it = 0; it < limit; ++it) {
         uint32_t done;
         asm volatile(
             "{\n\t.reg .pred p;\n\t"
@@ -432,6 +441,7 @@ __global__ void __launch_bounds__(kTcThreads + 32, 1) fluxbin_tc_kernel(const Tc
         // ---- issuer: one thread issues every unit's MMAs in order ----
         if (lane == 0) {
             uint32_t fills0 = 0u, fills1 = 0u;   // completed fills of each buffer seen so far
+            uint32_t issued0 = 0u, issued1 = 0u; // commits issued on each buffer
             int g = 0;
             for (int item = blockIdx.x; item < a.n_items && ok; item += gridDim.x) {
                 const TcItem it = tc_item(a, item, U);
@@ -440,7 +450,7 @@ __global__ void __launch_bounds__(kTcThreads + 32, 1) fluxbin_tc_kernel(const Tc
                     const int bf = g & 1;
                     const bool br1 = NB1 > 0 && u >= U0;
                     const uint32_t f = bf ? fills1 : fills0;
-                    ok = tc_mbar_wait(full0 + 8u * bf, f & 1);
+                    ok = tc_mbar_wait(full0 + 8u * bf, f & 1, a.spin_limit);
                     if (bf) fills1 += 1;
                     else fills0 += 1;
                     if (!ok) break;
@@ -456,9 +466,21 @@ __global__ void __launch_bounds__(kTcThreads + 32, 1) fluxbin_tc_kernel(const Tc
                         first0 = false;
                     }
                     tc_commit(empty0 + 8u * bf);
+                    if (bf) issued1 += 1;
+                    else issued0 += 1;
                 }
             }
             if (!ok) atomicOr(a.err, 1u);
+            // Every MMA this thread issued must have finished before the
+            // accumulators are released, whatever happened to the waits above:
+            // wait (bounded, with the full limit) for the last commit on each
+            // buffer.  Only a tensor core that stopped answering leaves this
+            // undrained; the tensor memory is then kept rather than freed
+            // under running MMAs.
+            bool drained = true;
+            if (issued0 > 0) drained = tc_mbar_wait(empty0, (issued0 - 1) & 1, kTcSpinLimit) && drained;
+            if (issued1 > 0) drained = tc_mbar_wait(empty0 + 8, (issued1 - 1) & 1, kTcSpinLimit) && drained;
+            smem_at<uint32_t>(kTcBarOff + 36) = drained ? 1u : 0u;
         }
         __syncwarp();
     } else {
@@ -507,7 +529,7 @@ __global__ void __launch_bounds__(kTcThreads + 32, 1) fluxbin_tc_kernel(const Tc
                 const int par = (u - u_begin) & 1;
                 const bool br1 = NB1 > 0 && u >= U0;
                 const uint32_t cb = bf ? commits1 : commits0;
-                if (cb > 0 && ok) ok = tc_mbar_wait(empty0 + 8u * bf, (cb - 1) & 1);
+                if (cb > 0 && ok) ok = tc_mbar_wait(empty0 + 8u * bf, (cb - 1) & 1, a.spin_limit);
                 const uint32_t abuf = sb + kTcAOff + (uint32_t)bf * kTcABytes;
                 const uint32_t bbuf = sb + kTcBOff + (uint32_t)bf * kTcBBytes;
                 const uint2 cur = par ? wq[1] : wq[0];
@@ -532,7 +554,7 @@ __global__ void __launch_bounds__(kTcThreads + 32, 1) fluxbin_tc_kernel(const Tc
                 fence_async_smem();
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) tc_mbar_arrive(full0 + 8u * bf);
+                if (lane == 0 && !a.test_stall) tc_mbar_arrive(full0 + 8u * bf);
                 if (bf) commits1 += 1;
                 else commits0 += 1;
             }
@@ -544,7 +566,7 @@ __global__ void __launch_bounds__(kTcThreads + 32, 1) fluxbin_tc_kernel(const Tc
             if (u_end > u_begin) {
                 const int lb = (g - 1) & 1;
                 const uint32_t cl = lb ? commits1 : commits0;
-                if (ok) ok = tc_mbar_wait(empty0 + 8u * lb, (cl - 1) & 1);
+                if (ok) ok = tc_mbar_wait(empty0 + 8u * lb, (cl - 1) & 1, a.spin_limit);
                 tc_fence_after();
                 const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * kLanes) << 16) + (uint32_t)(4 * quarter);
 #pragma unroll
@@ -600,20 +622,19 @@ __global__ void __launch_bounds__(kTcThreads + 32, 1) fluxbin_tc_kernel(const Tc
                 tc_worker_sync();   // s_last_tc is rewritten by the next item
             }
         }
-        if (!ok) {
-            if (tid == 0) atomicOr(a.err, 1u);
-            // give any MMA still in flight a last, bounded chance to finish
-            // before the accumulators are released
-            if (commits0 > 0) (void)tc_mbar_wait(empty0, (commits0 - 1) & 1);
-            if (commits1 > 0) (void)tc_mbar_wait(empty0 + 8, (commits1 - 1) & 1);
-        }
+        if (!ok && tid == 0) atomicOr(a.err, 1u);
     }
     tc_fence_before();
     __syncthreads();
     if (warp == 0) {
         tc_fence_after();
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTcTmemCols)
-                     : "memory");
+        // the issuer's drain result (written before the barrier above)
+        if (smem_at<const uint32_t>(kTcBarOff + 36) != 0u) {
+            asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTcTmemCols)
+                         : "memory");
+        } else if (lane == 0) {
+            atomicOr(a.err, 2u);
+        }
     }
 }
 

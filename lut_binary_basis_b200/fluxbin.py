@@ -22,6 +22,7 @@ FLAG_Y_FP32 = 2
 FLAG_EARLY_WEIGHTS = 4
 FLAG_PATH_LUT = 8
 FLAG_PATH_TC = 16
+FLAG_TEST_WAIT_TIMEOUT = 32
 
 STATUS = {0: "FLUXBIN_OK", -1: "FLUXBIN_ERR_INVALID_ARG", -2: "FLUXBIN_ERR_BAD_SHAPE",
           -3: "FLUXBIN_ERR_MISALIGNED", -4: "FLUXBIN_ERR_UNSUPPORTED", -5: "FLUXBIN_ERR_SMEM_BUDGET",

@@ -58,6 +58,10 @@ def _load():
             lib.oracle_lut_table_sym.argtypes = [P, i32, P]
             lib.oracle_lut_lookup_sym.argtypes = [P, i32, i64]
             lib.oracle_lut_lookup_sym.restype = ctypes.c_double
+            lib.oracle_rebuild_rows.argtypes = [i64, i64, i32, i32, P, P, P, i32, i64, i32, P, P, P, P, i64, P, P]
+            lib.oracle_rebuild_rows.restype = None
+            lib.oracle_gemv_rows.argtypes = [i64, i64, P, i32, P, P]
+            lib.oracle_gemv_rows.restype = None
             lib.oracle_num_threads.restype = i32
             lib.oracle_set_num_threads.argtypes = [i32]
             _lib = lib
@@ -119,6 +123,32 @@ def linear(layer, x, rows: Optional[Sequence[int]] = None) -> np.ndarray:
     _load().oracle_linear_rows(L["M"], L["N"], L["Kb"], L["G"], _ptr(L["signs"]), _ptr(L["r"]), _ptr(L["c"]),
                                L["Ks"], L["n_sal"], L["Gs"], _ptr(L["sal_signs"]), _ptr(L["rs"]), _ptr(L["cs"]),
                                _ptr(L["sal_idx"]), B, _ptr(xx), rr.size, _ptr(rr), _ptr(y))
+    return y
+
+
+def rebuild_rows(layer, rows: Optional[Sequence[int]] = None) -> np.ndarray:
+    """Rows of W = sum_k diag(r_k) B_k diag(c_k) (+ the salient branch at its
+    true columns), rebuilt in fp64: float64 [len(rows)][N]."""
+    L = _unpack(layer)
+    rr = _rows(L["M"], rows)
+    W = np.zeros((rr.size, L["N"]), np.float64)
+    if rr.size == 0 or L["N"] == 0:
+        return W
+    _load().oracle_rebuild_rows(L["M"], L["N"], L["Kb"], L["G"], _ptr(L["signs"]), _ptr(L["r"]), _ptr(L["c"]),
+                                L["Ks"], L["n_sal"], L["Gs"], _ptr(L["sal_signs"]), _ptr(L["rs"]), _ptr(L["cs"]),
+                                _ptr(L["sal_idx"]), rr.size, _ptr(rr), _ptr(W))
+    return W
+
+
+def gemv_rows(W: np.ndarray, x) -> np.ndarray:
+    """y[b][q] = W[q] . x[b] in fp64 for rows already rebuilt by rebuild_rows."""
+    W = np.ascontiguousarray(W, dtype=np.float64)
+    xx = _f64(x)
+    y = np.zeros((xx.shape[0], W.shape[0]), np.float64)
+    if W.size == 0 or xx.shape[0] == 0:
+        return y
+    assert xx.shape[1] == W.shape[1]
+    _load().oracle_gemv_rows(W.shape[1], W.shape[0], _ptr(W), xx.shape[0], _ptr(xx), _ptr(y))
     return y
 
 

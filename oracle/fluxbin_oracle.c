@@ -29,7 +29,7 @@
  * the column scale is fused into v (v = c (.) x), and a row's result is the
  * sum of the table entries that its sign patterns select, times the row scale.
  *
- * Readings where the pages are silent (each listed in the design notes):
+ * Readings where the pages are silent:
  *   bit value 1 means +1, 0 means -1; bit t of a pattern is column j*mu + t;
  *   the symmetric half table keeps the entries whose top bit (t = mu-1) is 0.
  */
@@ -81,6 +81,35 @@ static double row_scale(const double* r, int64_t M, int64_t N, int G, int k, int
  *   rows      [nrows]  row indices to evaluate
  *   y         [B][nrows]
  */
+/* Row i of W in fp64 (w has N entries). */
+static void rebuild_row(int64_t M, int64_t N, int Kb, int G,
+                        const int8_t* signs, const double* r, const double* c,
+                        int Ks, int64_t n_sal, int Gs,
+                        const int8_t* sal_signs, const double* rs, const double* cs,
+                        const int32_t* sal_idx, int64_t i, double* w) {
+    for (int64_t j = 0; j < N; ++j) w[j] = 0.0;
+    for (int k = 0; k < Kb; ++k) {
+        const int8_t* s = signs + ((int64_t)k * M + i) * N;
+        for (int64_t j = 0; j < N; ++j)
+            w[j] += row_scale(r, M, N, G, k, i, j) * (double)s[j] * c[(int64_t)k * N + j];
+    }
+    for (int k = 0; k < Ks; ++k) {
+        const int8_t* s = sal_signs + ((int64_t)k * M + i) * n_sal;
+        for (int64_t t = 0; t < n_sal; ++t)
+            w[sal_idx[t]] += row_scale(rs, M, n_sal, Gs, k, i, t) * (double)s[t] * cs[(int64_t)k * n_sal + t];
+    }
+}
+
+/* y[b] = w . x[b] for one rebuilt row. */
+static void dot_row(int64_t N, const double* w, int B, const double* x, int64_t nrows, int64_t q, double* y) {
+    for (int b = 0; b < B; ++b) {
+        const double* xb = x + (int64_t)b * N;
+        double acc = 0.0;
+        for (int64_t j = 0; j < N; ++j) acc += w[j] * xb[j];
+        y[(int64_t)b * nrows + q] = acc;
+    }
+}
+
 void oracle_linear_rows(int64_t M, int64_t N, int Kb, int G,
                         const int8_t* signs, const double* r, const double* c,
                         int Ks, int64_t n_sal, int Gs,
@@ -93,27 +122,30 @@ void oracle_linear_rows(int64_t M, int64_t N, int Kb, int G,
         double* w = (double*)malloc(sizeof(double) * (size_t)(N > 0 ? N : 1));
         #pragma omp for schedule(static)
         for (int64_t q = 0; q < nrows; ++q) {
-            int64_t i = rows[q];
-            for (int64_t j = 0; j < N; ++j) w[j] = 0.0;
-            for (int k = 0; k < Kb; ++k) {
-                const int8_t* s = signs + ((int64_t)k * M + i) * N;
-                for (int64_t j = 0; j < N; ++j)
-                    w[j] += row_scale(r, M, N, G, k, i, j) * (double)s[j] * c[(int64_t)k * N + j];
-            }
-            for (int k = 0; k < Ks; ++k) {
-                const int8_t* s = sal_signs + ((int64_t)k * M + i) * n_sal;
-                for (int64_t t = 0; t < n_sal; ++t)
-                    w[sal_idx[t]] += row_scale(rs, M, n_sal, Gs, k, i, t) * (double)s[t] * cs[(int64_t)k * n_sal + t];
-            }
-            for (int b = 0; b < B; ++b) {
-                const double* xb = x + (int64_t)b * N;
-                double acc = 0.0;
-                for (int64_t j = 0; j < N; ++j) acc += w[j] * xb[j];
-                y[(int64_t)b * nrows + q] = acc;
-            }
+            rebuild_row(M, N, Kb, G, signs, r, c, Ks, n_sal, Gs, sal_signs, rs, cs, sal_idx, rows[q], w);
+            dot_row(N, w, B, x, nrows, q, y);
         }
         free(w);
     }
+}
+
+/* The two halves of oracle_linear_rows, timed apart by the CPU baseline:
+ * the requested rows of W rebuilt in fp64 (W [nrows][N]) ... */
+void oracle_rebuild_rows(int64_t M, int64_t N, int Kb, int G,
+                         const int8_t* signs, const double* r, const double* c,
+                         int Ks, int64_t n_sal, int Gs,
+                         const int8_t* sal_signs, const double* rs, const double* cs,
+                         const int32_t* sal_idx,
+                         int64_t nrows, const int64_t* rows, double* W) {
+    #pragma omp parallel for schedule(static)
+    for (int64_t q = 0; q < nrows; ++q)
+        rebuild_row(M, N, Kb, G, signs, r, c, Ks, n_sal, Gs, sal_signs, rs, cs, sal_idx, rows[q], W + q * N);
+}
+
+/* ... and the GEMV on those rebuilt rows: y[b][q] = W[q] . x[b]. */
+void oracle_gemv_rows(int64_t N, int64_t nrows, const double* W, int B, const double* x, double* y) {
+    #pragma omp parallel for schedule(static)
+    for (int64_t q = 0; q < nrows; ++q) dot_row(N, W + q * N, B, x, nrows, q, y);
 }
 
 /* All 2^mu signed partial sums of one sub-vector: T[p] = sum_t (2 bit_t(p) - 1) v_t. */

@@ -319,3 +319,25 @@ def test_zero_batch_and_zero_rows():
     d = make_layer(sp, [42])
     assert oracle.linear(d, np.zeros((0, 16), np.float16)).shape == (0, 8)
     assert oracle.linear(d, make_x(sp, 1, [43]), rows=[]).shape == (1, 0)
+
+
+def oracle_rebuild_then_gemv(d, x):
+    return oracle.gemv_rows(oracle.rebuild_rows(d), x)
+
+
+@pytest.mark.parametrize("pin", PINS, ids=lambda p: p.__name__)
+def test_rebuild_then_gemv_pins(pin):
+    """The CPU baseline's two timed halves (rows of W rebuilt in fp64, then the
+    GEMV on them) satisfy the same closed forms and invariants."""
+    pin(oracle_rebuild_then_gemv)
+
+
+def test_rebuilt_rows_are_columns_of_the_layer_map():
+    """Column j of the rebuilt W is the layer's response to the unit vector
+    e_j, and a subset of rows is the same rows of the full rebuild."""
+    d = make_layer(spec_of(37, 50, 2, 2, 9, G=10, Gs=3), [41])
+    W = oracle.rebuild_rows(d)
+    E = np.eye(50, dtype=np.float16)
+    assert np.array_equal(W.T, oracle.linear(d, E))
+    rows = [36, 0, 17]
+    assert np.array_equal(oracle.rebuild_rows(d, rows), W[rows])

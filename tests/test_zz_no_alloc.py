@@ -6,7 +6,10 @@ direct cudaMalloc, or a latency-critical loop that must never call
 cudaMalloc / cudaFree because they synchronise the device.
 fluxbin_linear_static_scratch serves them with a fixed scratch array inside
 the library.  This test calls it through the C-ABI, twice in a row, and
-checks each result against fluxbin_linear given a caller-allocated workspace.
+checks each result against the fp64 oracle and against fluxbin_linear given a
+caller-allocated workspace, on launch plans that reduce inside a cluster, not
+at all, through the scratch (LUT path) and on the tensor cores (whose split
+items reduce through the scratch too).
 
 The file name sorts last so that a run stopping at the first failure has
 already run every other test.
@@ -18,6 +21,7 @@ import pytest
 
 torch = pytest.importorskip("torch")
 
+import oracle  # noqa: E402
 from lut_binary_basis_b200 import fluxbin, synth  # noqa: E402
 from lut_binary_basis_b200.synth import LayerSpec  # noqa: E402
 
@@ -41,6 +45,7 @@ def close(got, ref, layer, x):
     (LayerSpec("ragged", 2100, 777, 2, 1, 40, 8), 3),
     (LayerSpec("mu4", 1500, 1030, 2, 2, 60, 4), 5),
     (LayerSpec("wide", 256, 65536, 2, 1, 300, 8), 2),   # reduction through the scratch
+    (LayerSpec("tc", 8192, 4096, 2, 1, 205, 8), 16),    # tensor cores, items reduced through the scratch
 ])
 def test_static_scratch_matches_workspace_entry_point(sp, B):
     if not torch.cuda.is_available():
@@ -55,6 +60,8 @@ def test_static_scratch_matches_workspace_entry_point(sp, B):
     d.linear(xd, y_ref, fluxbin.FLAG_Y_FP32, ws)
     torch.cuda.synchronize()
     ref = y_ref.cpu().numpy().astype(np.float64)
+    exact = oracle.linear(layer, x)
+    close(ref, exact, layer, x)
     for call in range(2):
         y = torch.full((B, sp.M), float("nan"), dtype=torch.float32, device="cuda")
         fluxbin.fluxbin_linear_static_scratch(d.desc, d.words, d.r, d.c, d.swords, d.rs, d.cs, d.idx, xd, B, y,
@@ -62,6 +69,7 @@ def test_static_scratch_matches_workspace_entry_point(sp, B):
         torch.cuda.synchronize()
         got = y.cpu().numpy().astype(np.float64)
         assert np.all(np.isfinite(got)), f"call {call}"
+        close(got, exact, layer, x)
         close(got, ref, layer, x)
 
 
