@@ -773,6 +773,36 @@ def run_stack(args, device=None, summary=False):
     return res
 
 
+def run_fit(args):
+    """Host decomposition fitting of a dense 4096 x 4096 matrix into the
+    2.75-bit stack layout (2 global bases with G = 128 row-scale blocks, 16
+    salient columns per 128-column block with 2 extra bases and one salient
+    row scale per 16 of them): the library's threaded C++ fitter against the
+    fp64 numpy oracle, same steps and iteration count.  W_ij = a_i b_j z_ij with
+    a, b ~ LogNormal(0, 0.5), z ~ N(0, 1), seeded."""
+    from lut_binary_basis_b200 import fluxbin
+    from oracle import fit as ofit
+    M = N = args.fit_size
+    g = np.random.default_rng(2024)
+    W = np.exp(0.5 * g.standard_normal(M))[:, None] * np.exp(0.5 * g.standard_normal(N))[None, :] * \
+        g.standard_normal((M, N))
+    S = np.concatenate([blk * 128 + np.sort(g.choice(128, 16, replace=False)) for blk in range(N // 128)])
+    S = S.astype(np.int32)
+    it = args.fit_iters
+    t0 = time.perf_counter()
+    res = fluxbin.fluxbin_fit_hybrid(W, 2, S, 2, 128, 16, it)
+    t_lib = time.perf_counter() - t0
+    out = {"metric": "host decomposition fitting time", "unit": "s", "M": M, "N": N, "Kb": 2, "G": 128, "Ks": 2,
+           "n_sal": int(S.size), "Gs": 16, "iters": it, "threads": os.cpu_count(), "cpu_model": cpu_model(),
+           "library_s": t_lib, "relative_error": math.sqrt(res[-1] / float(np.sum(W * W)))}
+    if not args.no_cpu:
+        t0 = time.perf_counter()
+        (gs, gr, gc), (ss, sr, sc) = ofit.fit_hybrid(W, S, 2, 2, 128, 16, it)
+        out["oracle_s"] = time.perf_counter() - t0
+        out["signs_equal"] = bool(np.array_equal(gs, res[0]) and np.array_equal(ss, res[3]))
+    return out
+
+
 def run_reference(args, rank, world):
     """The oracle (CPU, all host cores): every step is one full call (rows of W
     rebuilt from signs and scales, then W x) on the same bounded sample of the
@@ -830,6 +860,10 @@ def main(argv=None):
     ap.add_argument("--stack", action="store_true",
                     help="time the 32-layer LLaMA-2-7B-shaped stack of 2.75-bit linears instead")
     ap.add_argument("--stack-layers", type=int, default=32)
+    ap.add_argument("--fit", action="store_true",
+                    help="time the host decomposition fitter (library vs oracle) on a dense matrix instead")
+    ap.add_argument("--fit-size", type=int, default=4096)
+    ap.add_argument("--fit-iters", type=int, default=5)
     args = ap.parse_args(argv)
     args.warmup = max(3, args.warmup)
     rank, local_rank, world = dist_env()
@@ -838,6 +872,9 @@ def main(argv=None):
         return
     if args.stack:
         print(json.dumps(run_stack(args)), flush=True)
+        return
+    if args.fit:
+        print(json.dumps(run_fit(args)), flush=True)
         return
     if args.impl == "reference":
         res = run_reference(args, rank, world)

@@ -304,6 +304,71 @@ int fluxbin_linear_static_scratch(const fluxbin_layer_desc* desc,
                                   const int32_t* d_idx, const uint16_t* d_x, int32_t B,
                                   void* d_y, uint32_t flags, void* stream);
 
+/*
+ * ---------------------------------------------------------------------------
+ * Decomposition fitting (host, offline): from a dense W to bases and scales
+ * ---------------------------------------------------------------------------
+ * FluxBin summary, Section 3 "Parameter Optimization": the bases B_k and the
+ * scales r_k, c_k of one branch minimise the weighted reconstruction error
+ *     E = sum_ij h_j (W_ij - sum_k r_k(i,j) B_k[i][j] c_k[j])^2
+ * by alternating minimisation.  Appendix A.1: with the bases and the column
+ * scales fixed, each row scale (each row block's scale when G > 0) has the
+ * closed form sum_j h_j R_ij B_ij c_j / sum_j h_j c_j^2 over the residual R
+ * of the other bases; symmetrically each column scale is
+ * sum_i R_ij B_ij r_i / sum_i r_i^2.  Appendix A.2: with the scales fixed,
+ * every element independently takes the best of its 2^nbases sign
+ * combinations (exhaustive search, globally optimal for those scales).
+ *
+ * Procedure (fixed, so that results are reproducible):
+ *   start: for k = 0 .. nbases-1, B_k = sign of the residual of the bases
+ *          already placed (sign(0) = +1), c_k = 1, r_k by the row closed form;
+ *   then `iters` times: for k = 0 .. nbases-1 the row scales of base k, then
+ *          its column scales (the other bases fixed at their latest values);
+ *          then the joint sign search over all elements.
+ *   A scale whose denominator is zero is set to 0.  Among sign combinations
+ *   with equal error the lowest p wins (bit k of p set means +1).
+ * The error E never increases from one step to the next.  Work is spread over
+ * the host's threads; results do not depend on the thread count.  The scales
+ * are returned in fp64; round them to fp16 for the device entry points.
+ *
+ *   M, N           shape of W (M output rows, N input columns), >= 0
+ *   nbases         bases of the branch, 1..8
+ *   row_scale_group 0: r is [nbases][M]; G > 0: r is [nbases][ceil(N/G)][M]
+ *   iters          alternating iterations after the start, >= 0
+ *   W              host fp64 [M][N], row-major
+ *   col_weight     host fp64 [N], every entry >= 0 (the h_j above), or NULL for all 1
+ *   signs_out      host int8 [nbases][M][N], +1 / -1
+ *   r_out, c_out   host fp64, layouts as above; c is [nbases][N]
+ *   objective_out  host, the final E (may be NULL)
+ * All buffers are the caller's.  Host only; no CUDA call.
+ * Errors: INVALID_ARG (null array with M*N > 0), BAD_SHAPE (negative sizes or
+ * iters, a negative or NaN weight), UNSUPPORTED (nbases outside 1..8).
+ */
+int fluxbin_fit(int32_t M, int32_t N, int32_t nbases, int32_t row_scale_group, int32_t iters,
+                const double* W, const double* col_weight, int8_t* signs_out, double* r_out, double* c_out,
+                double* objective_out);
+
+/*
+ * The hybrid layer (FluxBin summary, Section 3 "Salient-Aware Hybrid Bases"):
+ * Kb global bases fitted to W as by fluxbin_fit, then Ks salient bases fitted
+ * by the same procedure to the global residual gathered at the salient
+ * columns S (a dense M x n_sal matrix -- the Virtual Columnar Mapping layout),
+ * with the weights h_{S[t]} and their own row-scale group Gs.  The outputs
+ * are the arrays fluxbin_pack and the device entry points take (after
+ * rounding the scales to fp16):
+ *   signs_out [Kb][M][N], r_out, c_out      as for fluxbin_fit
+ *   sal_signs_out [Ks][M][n_sal], rs_out ([Ks][M] or [Ks][ceil(n_sal/Gs)][M]), cs_out [Ks][n_sal]
+ *   sal_idx   host int32 [n_sal], strictly increasing, each in [0, N)
+ *   objective_out  E of the whole reconstruction (global + salient)
+ * With Ks == 0 or n_sal == 0 only the global branch is fitted (the salient
+ * arrays may be NULL).
+ * Errors: as fluxbin_fit; BAD_SHAPE for a bad salient column list.
+ */
+int fluxbin_fit_hybrid(int32_t M, int32_t N, int32_t Kb, int32_t row_scale_group, int32_t Ks, int32_t n_sal,
+                       const int32_t* sal_idx, int32_t sal_scale_group, int32_t iters, const double* W,
+                       const double* col_weight, int8_t* signs_out, double* r_out, double* c_out,
+                       int8_t* sal_signs_out, double* rs_out, double* cs_out, double* objective_out);
+
 #ifdef __cplusplus
 }
 #endif

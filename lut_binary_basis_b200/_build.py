@@ -23,7 +23,7 @@ NVCC_FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-Xcompil
 CXX_FLAGS = ["-O3", "-std=c++17", "-fPIC", "-Wall", "-pthread", "-I", os.path.join(ROOT, "include")]
 
 CU_SOURCES = ["fluxbin_api.cu", "fluxbin_inst_mu8.cu", "fluxbin_inst_mu4.cu", "fluxbin_inst_tc.cu"]
-CXX_SOURCES = ["fluxbin_pack.cpp"]
+CXX_SOURCES = ["fluxbin_pack.cpp", "fluxbin_fit.cpp"]
 
 
 def _nvcc() -> str:

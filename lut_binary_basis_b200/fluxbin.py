@@ -77,8 +77,11 @@ def lib():
             L.fluxbin_linear.argtypes = [P, P, P, P, P, P, P, P, P, i32, P, u32, P, sz, P]
             L.fluxbin_linear_static_scratch.argtypes = [P, P, P, P, P, P, P, P, P, i32, P, u32, P]
             L.fluxbin_device_status.argtypes = [ctypes.POINTER(u32)]
+            L.fluxbin_fit.argtypes = [i32, i32, i32, i32, i32, P, P, P, P, P, P]
+            L.fluxbin_fit_hybrid.argtypes = [i32, i32, i32, i32, i32, i32, P, i32, i32, P, P, P, P, P, P, P, P, P]
             for f in ("fluxbin_packed_sizes", "fluxbin_pack", "fluxbin_workspace_bytes", "fluxbin_lut_gemv",
-                      "fluxbin_linear", "fluxbin_linear_static_scratch", "fluxbin_device_status"):
+                      "fluxbin_linear", "fluxbin_linear_static_scratch", "fluxbin_device_status", "fluxbin_fit",
+                      "fluxbin_fit_hybrid"):
                 getattr(L, f).restype = ctypes.c_int
             _lib = L
     return _lib
@@ -184,6 +187,48 @@ def fluxbin_linear_static_scratch(desc: LayerDesc, words, r, c, swords, rs, cs, 
     _check(lib().fluxbin_linear_static_scratch(ctypes.byref(desc), _dptr(words), _dptr(r), _dptr(c), _dptr(swords),
                                                _dptr(rs), _dptr(cs), _dptr(idx), _dptr(x), B, _dptr(y), flags,
                                                _stream(stream)), "fluxbin_linear_static_scratch")
+
+
+def _scale_shape(nb: int, M: int, ncols: int, G: int):
+    return (nb, -(-ncols // G), M) if G > 0 else (nb, M)
+
+
+def fluxbin_fit(W: np.ndarray, nbases: int, row_scale_group: int = 0, iters: int = 10,
+                col_weight: Optional[np.ndarray] = None):
+    """Host decomposition fitting of one branch (include/fluxbin.h): returns
+    (signs int8 [nb][M][N], r fp64, c fp64 [nb][N], objective)."""
+    W = np.ascontiguousarray(W, dtype=np.float64)
+    M, N = W.shape
+    h = None if col_weight is None else np.ascontiguousarray(col_weight, dtype=np.float64)
+    signs = np.zeros((nbases, M, N), np.int8)
+    r = np.zeros(_scale_shape(nbases, M, N, row_scale_group), np.float64)
+    c = np.zeros((nbases, N), np.float64)
+    obj = ctypes.c_double()
+    _check(lib().fluxbin_fit(M, N, nbases, row_scale_group, iters, _np_ptr(W), _np_ptr(h), _np_ptr(signs),
+                             _np_ptr(r), _np_ptr(c), ctypes.byref(obj)), "fluxbin_fit")
+    return signs, r, c, obj.value
+
+
+def fluxbin_fit_hybrid(W: np.ndarray, Kb: int, sal_idx: np.ndarray, Ks: int, row_scale_group: int = 0,
+                       sal_scale_group: int = 0, iters: int = 10, col_weight: Optional[np.ndarray] = None):
+    """Global bases, then the salient refinement on the residual at columns
+    sal_idx: returns (signs, r, c, sal_signs, rs, cs, objective)."""
+    W = np.ascontiguousarray(W, dtype=np.float64)
+    M, N = W.shape
+    idx = np.ascontiguousarray(sal_idx, dtype=np.int32)
+    ns = int(idx.size) if Ks else 0
+    h = None if col_weight is None else np.ascontiguousarray(col_weight, dtype=np.float64)
+    signs = np.zeros((Kb, M, N), np.int8)
+    r = np.zeros(_scale_shape(Kb, M, N, row_scale_group), np.float64)
+    c = np.zeros((Kb, N), np.float64)
+    ss = np.zeros((Ks, M, ns), np.int8)
+    rs = np.zeros(_scale_shape(Ks, M, ns, sal_scale_group), np.float64)
+    cs = np.zeros((Ks, ns), np.float64)
+    obj = ctypes.c_double()
+    _check(lib().fluxbin_fit_hybrid(M, N, Kb, row_scale_group, Ks, ns, _np_ptr(idx), sal_scale_group, iters,
+                                    _np_ptr(W), _np_ptr(h), _np_ptr(signs), _np_ptr(r), _np_ptr(c), _np_ptr(ss),
+                                    _np_ptr(rs), _np_ptr(cs), ctypes.byref(obj)), "fluxbin_fit_hybrid")
+    return signs, r, c, ss, rs, cs, obj.value
 
 
 def pack_host(layer) -> dict:
