@@ -374,7 +374,7 @@ def layer_entry(spec, layer, B, device, l2, wid, steps=50, path_flags=0):
     import torch
     from lut_binary_basis_b200 import fluxbin
     copies, xs, ys, R = build_pool(layer, spec, B, device, l2, wid)
-    ws = fluxbin.new_workspace(spec.M, B, device)
+    ws = copies[0].workspace(B)
     flags = fluxbin.FLAG_EARLY_WEIGHTS | path_flags
     stream = torch.cuda.Stream(device)
     g = capture_rotation(copies, xs, ys, ws, flags, stream)
@@ -471,7 +471,7 @@ def run_ours(args, rank, local_rank, world):
     props = torch.cuda.get_device_properties(device)
     l2 = getattr(props, "L2_cache_size", 126 * 2 ** 20) or 126 * 2 ** 20
     copies, xs, ys, R = build_pool(layer, spec, B, device, l2, HEADLINE_WID)
-    ws = fluxbin.new_workspace(spec.M, B, device)
+    ws = copies[0].workspace(B)
     flags = fluxbin.FLAG_EARLY_WEIGHTS  # fp16 y
 
     stream = torch.cuda.Stream(device)
@@ -725,7 +725,7 @@ def run_stack(args, device=None, summary=False):
         torch.cuda.set_device(device)
     layers = build_stack(device, n_layers, workers)
     setup_s = time.time() - t0
-    ws = fluxbin.new_workspace(max(sp.M for sp, *_ in layers), 1, device)
+    ws = max((dl.workspace(1) for _, dl, _, _ in layers), key=lambda t: t.numel())
     flags = fluxbin.FLAG_EARLY_WEIGHTS
     stream = torch.cuda.Stream(device)
 

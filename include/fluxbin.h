@@ -136,6 +136,13 @@ typedef struct fluxbin_layer_desc {
 #define FLUXBIN_FLAG_PATH_LUT     8u  /* always use the LUT path */
 #define FLUXBIN_FLAG_PATH_TC      16u /* always use the tensor-core path (UNSUPPORTED when the layer
                                          does not qualify, WORKSPACE without a workspace) */
+#define FLUXBIN_FLAG_SEPARATE_TABLES 64u /* batch 1, mu = 8, per-row scales: build every unit's tables
+                                         once in a kernel of its own (the precompute as a separate
+                                         operator) and look them up from shared-memory copies of the
+                                         table buffer; needs fluxbin_layer_workspace_bytes() of
+                                         workspace (WORKSPACE otherwise), UNSUPPORTED for other
+                                         layers, INVALID_ARG with FLUXBIN_FLAG_PATH_TC.  Measured
+                                         slower than the default on B200 (see the batch-1 kernels). */
 #define FLUXBIN_FLAG_TEST_WAIT_TIMEOUT 32u /* test hook, only together with FLUXBIN_FLAG_PATH_TC: the
                                          tensor-core kernel's preparing warps never report a buffer
                                          ready and every wait gives up after a few polls, so the
@@ -224,6 +231,27 @@ int fluxbin_pack(const fluxbin_layer_desc* desc, const int8_t* signs, const int8
 int fluxbin_workspace_bytes(int32_t M, int32_t B, size_t* bytes);
 
 /*
+ * Workspace for one layer at batch B, in bytes: fluxbin_workspace_bytes(M, B)
+ * plus, for a layer whose batch-1 calls can run the table precompute as a
+ * separate kernel (B == 1, mu == 8, per-row scales in both branches), a table
+ * buffer of 64 KiB per pair of units (a unit is (32/nb)*mu columns of a
+ * branch).  Host only.
+ *
+ * With FLUXBIN_FLAG_SEPARATE_TABLES and at least this many bytes, a batch-1
+ * mu = 8 call builds every unit's tables of signed partial sums once, in a
+ * kernel of its own that writes them to the table buffer (the precompute as
+ * a separate operator, LUT Tensor Core notes, Section 3.1.1), and the lookup
+ * kernel copies each unit's tables into shared memory with bulk copies
+ * instead of rebuilding them in every CTA.  Without the flag the tables are
+ * built inside the lookup kernel.  Both give the same results up to fp32
+ * summation order.  The first fluxbin_workspace_bytes(M, B) bytes keep the
+ * zero-fill contract of fluxbin_workspace_bytes; the table buffer after them
+ * holds scratch and needs no initialisation.
+ * Errors: INVALID_ARG (null desc or output), BAD_SHAPE, UNSUPPORTED.
+ */
+int fluxbin_layer_workspace_bytes(const fluxbin_layer_desc* desc, int32_t B, size_t* bytes);
+
+/*
  * One dense branch (the kernel that Virtual Columnar Mapping reuses):
  *   y[b][i] (+)= sum_k r_k(i) * sum_{n < ncols} B_k[i][n] c_k[n] x[b][col(n)]
  * with col(n) = d_gather[n] (or n when d_gather is NULL).
@@ -237,8 +265,9 @@ int fluxbin_workspace_bytes(int32_t M, int32_t B, size_t* bytes);
  *   d_x          fp16 [B][N];  B in [0, 16]
  *   d_y          [B][M], fp16 or fp32 per FLUXBIN_FLAG_Y_FP32; 4-byte aligned for fp32
  *   flags        FLUXBIN_FLAG_*
- *   d_workspace, workspace_bytes   see fluxbin_workspace_bytes (may be NULL/0 only
- *                when that function reports fewer bytes than given)
+ *   d_workspace, workspace_bytes   see fluxbin_workspace_bytes (may be NULL/0 only when
+ *                the call needs none; FLUXBIN_FLAG_SEPARATE_TABLES needs
+ *                fluxbin_workspace_bytes(M, 1) + 64 KiB per pair of units)
  * M == 0 or B == 0 returns FLUXBIN_OK without launching.
  * Errors: INVALID_ARG, BAD_SHAPE, MISALIGNED, UNSUPPORTED, SMEM_BUDGET, WORKSPACE, CUDA.
  */

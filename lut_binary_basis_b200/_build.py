@@ -22,7 +22,8 @@ NVCC_FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-Xcompil
               "--expt-relaxed-constexpr", "-I", os.path.join(ROOT, "include")] + ARCH
 CXX_FLAGS = ["-O3", "-std=c++17", "-fPIC", "-Wall", "-pthread", "-I", os.path.join(ROOT, "include")]
 
-CU_SOURCES = ["fluxbin_api.cu", "fluxbin_inst_mu8.cu", "fluxbin_inst_mu4.cu", "fluxbin_inst_tc.cu"]
+CU_SOURCES = ["fluxbin_api.cu", "fluxbin_inst_mu8.cu", "fluxbin_inst_mu4.cu", "fluxbin_inst_tc.cu",
+              "fluxbin_inst_lut1.cu", "fluxbin_inst_lut1h.cu"]
 CXX_SOURCES = ["fluxbin_pack.cpp", "fluxbin_fit.cpp"]
 
 

@@ -24,6 +24,17 @@ KernelFn select_kernel_mu4(int nb0, int nb1, int bt, int gs1);
 KernelFn select_kernel_mu8_3(int nb0, int nb1, int bt, int gs1);
 using TcKernelFn = void (*)(TcArgs);
 TcKernelFn select_tc_kernel(int mu, int nb0, int nb1);
+KernelFn select_kernel_lut1(int lw, int nb0, int nb1);
+using TabKernelFn = void (*)(KernelArgs, float*);
+using HKernelFn = void (*)(KernelArgs, const float*);
+TabKernelFn select_tables_kernel(int nb0, int nb1);
+HKernelFn select_kernel_lut1h(int spw, int nb0, int nb1);
+int lut1h_threads(int spw);
+int lut1h_smem_bytes(int spw);
+int lut1h_slabs(int spw);
+int lut1_threads(int lw);
+int lut1_smem_bytes(int lw);
+int lut1_slabs(int lw);
 
 // Automatic path choice for a layer both paths can run.  Measured on B200
 // (µs per call, LUT / tensor cores): 4096x4096 B=8 17.6/35.7, B=16 31.0/38.1;
@@ -76,6 +87,15 @@ struct FuncInfo {
     int blocks_per_sm = 0;  // with the reduction buffer
 };
 
+// CTA shape of a kernel for the planner: row slabs per CTA, threads, dynamic
+// shared memory.
+struct CtaShape {
+    int slabs;
+    int threads;
+    size_t smem;
+};
+
+
 std::mutex g_mu;
 std::unordered_map<int, DeviceInfo> g_dev;
 std::unordered_map<uint64_t, FuncInfo> g_func;
@@ -98,7 +118,7 @@ int device_info(int dev, DeviceInfo* out) {
 
 // Per-function, per-device set-up: opt in to the dynamic shared memory of the
 // largest launch and to non-portable cluster sizes; occupancy.
-int func_info(KernelFn fn, int dev, int mu, int bt, int gs1, const DeviceInfo& di, FuncInfo* out) {
+int func_info_shape(KernelFn fn, int dev, size_t smem_max, int threads, const DeviceInfo& di, FuncInfo* out) {
     const uint64_t key = (reinterpret_cast<uint64_t>(fn) << 8) ^ (uint64_t)dev;
     auto it = g_func.find(key);
     if (it != g_func.end()) {
@@ -106,7 +126,6 @@ int func_info(KernelFn fn, int dev, int mu, int bt, int gs1, const DeviceInfo& d
         return FLUXBIN_OK;
     }
     FuncInfo fi;
-    const size_t smem_max = table_smem_bytes(mu, bt) + red_smem_bytes(bt) + scale_smem_bytes(gs1);
     cudaFuncAttributes fa;
     cudaError_t e = cudaFuncGetAttributes(&fa, fn);
     if (e != cudaSuccess) return cuda_fail(e);
@@ -114,7 +133,7 @@ int func_info(KernelFn fn, int dev, int mu, int bt, int gs1, const DeviceInfo& d
     if ((size_t)di.max_smem < smem_max + fa.sharedSizeBytes) return FLUXBIN_ERR_SMEM_BUDGET;
     if ((e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_max)) != cudaSuccess ||
         (e = cudaFuncSetAttribute(fn, cudaFuncAttributeNonPortableClusterSizeAllowed, 1)) != cudaSuccess ||
-        (e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&fi.blocks_per_sm, fn, kThreads, smem_max)) != cudaSuccess)
+        (e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&fi.blocks_per_sm, fn, threads, smem_max)) != cudaSuccess)
         return cuda_fail(e);
     if (fi.blocks_per_sm < 1) return FLUXBIN_ERR_SMEM_BUDGET;
     g_func.emplace(key, fi);
@@ -122,14 +141,23 @@ int func_info(KernelFn fn, int dev, int mu, int bt, int gs1, const DeviceInfo& d
     return FLUXBIN_OK;
 }
 
+int func_info(KernelFn fn, int dev, int mu, int bt, int gs1, const DeviceInfo& di, FuncInfo* out) {
+    return func_info_shape(fn, dev, table_smem_bytes(mu, bt) + red_smem_bytes(bt) + scale_smem_bytes(gs1), kThreads,
+                           di, out);
+}
+
+CtaShape v1_shape(int mu, int bt, int gs1) {
+    return CtaShape{kSlabsPerCta, kThreads, table_smem_bytes(mu, bt) + red_smem_bytes(bt) + scale_smem_bytes(gs1)};
+}
+
 // How many clusters of `csize` CTAs can be resident at once (0: none).
-int max_active_clusters(KernelFn fn, int dev, int csize, size_t smem) {
+int max_active_clusters(KernelFn fn, int dev, int csize, size_t smem, int threads = kThreads) {
     const uint64_t key = (reinterpret_cast<uint64_t>(fn) << 12) ^ ((uint64_t)dev << 8) ^ (uint64_t)csize;
     auto it = g_clusters.find(key);
     if (it != g_clusters.end()) return it->second;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)csize);
-    cfg.blockDim = dim3(kThreads);
+    cfg.blockDim = dim3((unsigned)threads);
     cfg.dynamicSmemBytes = smem;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -171,16 +199,16 @@ struct Plan {
 // SM: one CTA's table build then overlaps the other's lookups).  When that
 // leaves most SMs idle (few rows, long rows) the units are split as widely
 // as the SMs allow and reduced through the workspace.
-Plan make_plan(KernelFn fn, int dev, int mu, int bt, int gs1, int64_t Ms, int64_t U, int n_bc,
-               const DeviceInfo& di, const FuncInfo& fi, bool have_ws) {
+Plan make_plan(KernelFn fn, int dev, const CtaShape& cs, int64_t Ms, int64_t U, int n_bc, const DeviceInfo& di,
+               const FuncInfo& fi, bool have_ws, bool fill_gpu = false) {
     Plan p;
-    p.n_rg = (int)((Ms + kSlabsPerCta - 1) / kSlabsPerCta);
+    p.n_rg = (int)((Ms + cs.slabs - 1) / cs.slabs);
     const int64_t groups = (int64_t)p.n_rg * n_bc;
     const int64_t slots = (int64_t)di.sm_count * fi.blocks_per_sm;
     int64_t want = slots / groups;
     if (want > U) want = U;
     if (want > kMaxCluster) want = kMaxCluster;
-    const size_t smem = table_smem_bytes(mu, bt) + red_smem_bytes(bt) + scale_smem_bytes(gs1);
+    const size_t smem = cs.smem;
     // Long rows on few row groups: a split wider than a cluster, reduced
     // through the workspace, shortens each CTA's chain of units by more than
     // the workspace reduction costs once a cluster would leave every CTA at
@@ -199,15 +227,24 @@ Plan make_plan(KernelFn fn, int dev, int mu, int bt, int gs1, int64_t Ms, int64_
         return p;
     }
     for (int64_t ks = want; ks >= 2; --ks) {
-        if (groups * ks * 2 < di.sm_count) break;  // too few CTAs: use the workspace instead
-        if (max_active_clusters(fn, dev, (int)ks, smem) >= groups) {
+        if (have_ws && groups * ks * 2 < di.sm_count) break;  // too few CTAs: use the workspace instead
+        if (max_active_clusters(fn, dev, (int)ks, smem, cs.threads) >= groups) {
             p.n_ks = (int)ks;
             p.cluster = true;
+            // One CTA per SM: a cluster size that fits fewer CTAs than the
+            // GPU has slots (clusters must sit inside one GPU processing
+            // cluster) leaves SMs idle; split one CTA per slot through the
+            // workspace instead when that fills at least an eighth more.
+            const int64_t ks_ws = std::min<int64_t>(U, slots / groups);
+            if (fill_gpu && have_ws && ks_ws * 8 >= ks * 9) {
+                p.n_ks = (int)ks_ws;
+                p.cluster = false;
+            }
             return p;
         }
     }
-    if (groups * 2 >= di.sm_count || U <= 1) {
-        p.n_ks = 1;  // enough row groups: no split at all
+    if (groups * 2 >= di.sm_count || U <= 1 || !have_ws) {
+        p.n_ks = 1;  // enough row groups (or no workspace): no split at all
         return p;
     }
     int64_t ks = (slots + groups / 2) / groups;
@@ -332,14 +369,220 @@ int run_tc(int32_t M, int32_t N, int mu, const BranchIn& g, const BranchIn* s, i
     return FLUXBIN_OK;
 }
 
+// Branch arguments of a launch.
+void fill_branches(KernelArgs& a, int mu, const BranchIn& g, const BranchIn* s, int nb1) {
+    const BranchIn* in[2] = {&g, nb1 ? s : nullptr};
+    for (int q = 0; q < 2; ++q) {
+        BranchArgs& o = a.br[q];
+        if (!in[q] || in[q]->ncols == 0) continue;
+        o.words = reinterpret_cast<const uint4*>(in[q]->words);
+        o.r = reinterpret_cast<const __half*>(in[q]->r);
+        o.c = reinterpret_cast<const __half*>(in[q]->c);
+        o.gather = in[q]->gather;
+        o.ncols = in[q]->ncols;
+        o.units = (int32_t)branch_units(in[q]->ncols, in[q]->nb, mu);
+        o.rgroup = in[q]->rgroup;
+        o.ngroups = in[q]->rgroup > 0 ? (in[q]->ncols + in[q]->rgroup - 1) / in[q]->rgroup : 0;
+    }
+}
+
+// Batch 1, mu = 8, per-row scales: the warp-specialised kernel
+// (fluxbin_lut1.cuh).  16 lookup warps per CTA (1024 rows, one CTA per SM)
+// when that plan keeps most SMs busy, else 8 (512 rows, two CTAs per SM).
+int run_lut1(int32_t M, int32_t N, const BranchIn& g, const BranchIn* s, int nb1, const uint16_t* d_x, void* d_y,
+             uint32_t flags, void* ws, size_t ws_bytes, void* stream, int* uses_ws) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return FLUXBIN_ERR_CUDA;
+    KernelArgs a = {};
+    fill_branches(a, 8, g, s, nb1);
+    a.Ms = (int32_t)row_slabs(M);
+    const int64_t U = (int64_t)a.br[0].units + a.br[1].units;
+    const bool have_ws = ws && ws_bytes >= workspace_bytes_for(M, 1) && aligned(ws, 16);
+    DeviceInfo di;
+    unsigned int* err = nullptr;
+    KernelFn fn = nullptr;
+    Plan plan;
+    int lw = 16;
+    {
+        std::lock_guard<std::mutex> lock(g_mu);
+        int st = device_info(dev, &di);
+        if (st != FLUXBIN_OK) return st;
+        KernelFn f16 = select_kernel_lut1(16, g.nb, nb1), f8 = select_kernel_lut1(8, g.nb, nb1);
+        if (!f16 || !f8) return FLUXBIN_ERR_UNSUPPORTED;
+        FuncInfo i16, i8;
+        const CtaShape c16{lut1_slabs(16), lut1_threads(16), (size_t)lut1_smem_bytes(16)};
+        const CtaShape c8{lut1_slabs(8), lut1_threads(8), (size_t)lut1_smem_bytes(8)};
+        if ((st = func_info_shape(f16, dev, c16.smem, c16.threads, di, &i16)) != FLUXBIN_OK) return st;
+        if ((st = func_info_shape(f8, dev, c8.smem, c8.threads, di, &i8)) != FLUXBIN_OK) return st;
+        const Plan p16 = make_plan(f16, dev, c16, a.Ms, U, 1, di, i16, have_ws, true);
+        const Plan p8 = make_plan(f8, dev, c8, a.Ms, U, 1, di, i8, have_ws);
+        const int64_t busy16 = (int64_t)p16.n_rg * p16.n_ks;   // CTAs = SMs in use
+        if (busy16 * 4 >= (int64_t)di.sm_count * 3) {
+            fn = f16;
+            plan = p16;
+        } else {
+            fn = f8;
+            plan = p8;
+            lw = 8;
+        }
+    }
+    {
+        std::lock_guard<std::mutex> lock(g_tc_mu);
+        const int st = device_error_address(dev, &err);
+        if (st != FLUXBIN_OK) return st;
+    }
+    a.x = reinterpret_cast<const __half*>(d_x);
+    a.y = d_y;
+    a.M = M;
+    a.N = N;
+    a.B = 1;
+    a.Mp = a.Ms * kLanes;
+    a.n_rg = plan.n_rg;
+    a.n_bc = 1;
+    a.n_ks = plan.n_ks;
+    a.cluster = plan.cluster ? 1 : 0;
+    a.flags = flags;
+    a.err = err;
+    if (uses_ws) {  // plan query only
+        *uses_ws = (a.n_ks > 1 && !plan.cluster) ? 1 : 0;
+        return FLUXBIN_OK;
+    }
+    if (a.n_ks > 1 && !plan.cluster) {
+        if (!have_ws) return ws ? (aligned(ws, 16) ? FLUXBIN_ERR_WORKSPACE : FLUXBIN_ERR_MISALIGNED)
+                                : FLUXBIN_ERR_WORKSPACE;
+        const size_t acc = (((size_t)a.Mp * sizeof(float)) + 255) & ~(size_t)255;
+        a.ws_acc = static_cast<float*>(ws);
+        a.ws_cnt = reinterpret_cast<unsigned int*>(static_cast<char*>(ws) + acc);
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)((int64_t)a.n_rg * a.n_ks));
+    cfg.blockDim = dim3((unsigned)lut1_threads(lw));
+    cfg.dynamicSmemBytes = (size_t)lut1_smem_bytes(lw);
+    cfg.stream = static_cast<cudaStream_t>(stream);
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (plan.cluster) {
+        attr[1].id = cudaLaunchAttributeClusterDimension;
+        attr[1].val.clusterDim.x = (unsigned)a.n_ks;
+        attr[1].val.clusterDim.y = 1;
+        attr[1].val.clusterDim.z = 1;
+        cfg.numAttrs = 2;
+    }
+    const cudaError_t le = cudaLaunchKernelEx(&cfg, fn, a);
+    if (le != cudaSuccess) return cuda_fail(le);
+    return FLUXBIN_OK;
+}
+
+// Batch 1, mu = 8, per-row scales, with room for the table buffer in the
+// workspace: the table precompute as its own kernel (fluxbin_tables.cuh),
+// then the lookups on the precomputed tables (fluxbin_lut1h.cuh).  2048 rows
+// per CTA when that plan keeps most SMs busy, else 1024.
+int run_lut1h(int32_t M, int32_t N, const BranchIn& g, const BranchIn* s, int nb1, const uint16_t* d_x, void* d_y,
+              uint32_t flags, void* ws, void* stream, int* uses_ws) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return FLUXBIN_ERR_CUDA;
+    KernelArgs a = {};
+    fill_branches(a, 8, g, s, nb1);
+    a.Ms = (int32_t)row_slabs(M);
+    const int64_t U = (int64_t)a.br[0].units + a.br[1].units;
+    DeviceInfo di;
+    unsigned int* err = nullptr;
+    HKernelFn fn = nullptr;
+    TabKernelFn tfn = select_tables_kernel(g.nb, nb1);
+    Plan plan;
+    int spw = 4;
+    {
+        std::lock_guard<std::mutex> lock(g_mu);
+        int st = device_info(dev, &di);
+        if (st != FLUXBIN_OK) return st;
+        HKernelFn f4 = select_kernel_lut1h(4, g.nb, nb1), f2 = select_kernel_lut1h(2, g.nb, nb1);
+        if (!f4 || !f2 || !tfn) return FLUXBIN_ERR_UNSUPPORTED;
+        FuncInfo i4, i2;
+        const CtaShape c4{lut1h_slabs(4), lut1h_threads(4), (size_t)lut1h_smem_bytes(4)};
+        const CtaShape c2{lut1h_slabs(2), lut1h_threads(2), (size_t)lut1h_smem_bytes(2)};
+        KernelFn k4 = reinterpret_cast<KernelFn>(f4), k2 = reinterpret_cast<KernelFn>(f2);
+        if ((st = func_info_shape(k4, dev, c4.smem, c4.threads, di, &i4)) != FLUXBIN_OK) return st;
+        if ((st = func_info_shape(k2, dev, c2.smem, c2.threads, di, &i2)) != FLUXBIN_OK) return st;
+        const Plan p4 = make_plan(k4, dev, c4, a.Ms, U, 1, di, i4, true, true);
+        const Plan p2 = make_plan(k2, dev, c2, a.Ms, U, 1, di, i2, true, true);
+        if ((int64_t)p4.n_rg * p4.n_ks * 4 >= (int64_t)di.sm_count * 3) {
+            fn = f4;
+            plan = p4;
+        } else {
+            fn = f2;
+            plan = p2;
+            spw = 2;
+        }
+    }
+    if (uses_ws) {  // plan query only: the tables always live in the workspace
+        *uses_ws = 1;
+        return FLUXBIN_OK;
+    }
+    {
+        std::lock_guard<std::mutex> lock(g_tc_mu);
+        const int st = device_error_address(dev, &err);
+        if (st != FLUXBIN_OK) return st;
+    }
+    a.x = reinterpret_cast<const __half*>(d_x);
+    a.y = d_y;
+    a.M = M;
+    a.N = N;
+    a.B = 1;
+    a.Mp = a.Ms * kLanes;
+    a.n_rg = plan.n_rg;
+    a.n_bc = 1;
+    a.n_ks = plan.n_ks;
+    a.cluster = plan.cluster ? 1 : 0;
+    a.flags = flags;
+    a.err = err;
+    const size_t acc = (((size_t)a.Mp * sizeof(float)) + 255) & ~(size_t)255;
+    a.ws_acc = static_cast<float*>(ws);
+    a.ws_cnt = reinterpret_cast<unsigned int*>(static_cast<char*>(ws) + acc);
+    float* tables = reinterpret_cast<float*>(static_cast<char*>(ws) + workspace_bytes_for(M, 1));
+
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t tc = {};
+    tc.gridDim = dim3((unsigned)((U + 1) / 2));
+    tc.blockDim = dim3(256);   // fluxbin_tables_kernel: one unit pair per CTA of 256 threads
+    tc.stream = static_cast<cudaStream_t>(stream);
+    tc.attrs = attr;
+    tc.numAttrs = 1;
+    cudaError_t le = cudaLaunchKernelEx(&tc, tfn, a, tables);
+    if (le != cudaSuccess) return cuda_fail(le);
+
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)((int64_t)a.n_rg * a.n_ks));
+    cfg.blockDim = dim3((unsigned)lut1h_threads(spw));
+    cfg.dynamicSmemBytes = (size_t)lut1h_smem_bytes(spw);
+    cfg.stream = static_cast<cudaStream_t>(stream);
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (plan.cluster) {
+        attr[1].id = cudaLaunchAttributeClusterDimension;
+        attr[1].val.clusterDim.x = (unsigned)a.n_ks;
+        attr[1].val.clusterDim.y = 1;
+        attr[1].val.clusterDim.z = 1;
+        cfg.numAttrs = 2;
+    }
+    le = cudaLaunchKernelEx(&cfg, fn, a, static_cast<const float*>(tables));
+    if (le != cudaSuccess) return cuda_fail(le);
+    return FLUXBIN_OK;
+}
+
 // Validates the arguments, chooses the path and the launch plan and launches
 // the layer.  With `uses_ws` non-null nothing is launched: it reports whether
 // the chosen plan reduces through the workspace.
 int run(int32_t M, int32_t N, int mu, const BranchIn& g, const BranchIn* s, const uint16_t* d_x, int32_t B,
         void* d_y, uint32_t flags, void* ws, size_t ws_bytes, void* stream, int* uses_ws = nullptr) {
     if (flags & ~(kFlagAccumulate | kFlagYFp32 | kFlagEarlyWeights | kFlagPathLut | kFlagPathTc |
-                  kFlagTestWaitTimeout))
+                  kFlagTestWaitTimeout | kFlagSeparateTables))
         return FLUXBIN_ERR_INVALID_ARG;
+    if ((flags & kFlagSeparateTables) && (flags & kFlagPathTc)) return FLUXBIN_ERR_INVALID_ARG;
     if ((flags & kFlagPathLut) && (flags & kFlagPathTc)) return FLUXBIN_ERR_INVALID_ARG;
     if ((flags & kFlagTestWaitTimeout) && !(flags & kFlagPathTc)) return FLUXBIN_ERR_INVALID_ARG;
     if (uses_ws) *uses_ws = 0;
@@ -362,16 +605,35 @@ int run(int32_t M, int32_t N, int mu, const BranchIn& g, const BranchIn* s, cons
     const bool tc_fits = (mu == 8 || mu == 4) && g.rgroup == 0 && (!nb1 || s->rgroup == 0);
     if ((flags & kFlagPathTc) && !tc_fits) return FLUXBIN_ERR_UNSUPPORTED;
     if ((flags & kFlagPathTc) ||
-        (!(flags & kFlagPathLut) && tc_fits && prefer_tensor_cores(M, N, B) && ws &&
+        (!(flags & (kFlagPathLut | kFlagSeparateTables)) && tc_fits && prefer_tensor_cores(M, N, B) && ws &&
          ws_bytes >= workspace_bytes_for(M, B)))
         return run_tc(M, N, mu, g, s, nb1, d_x, B, d_y, flags & ~(kFlagPathLut | kFlagPathTc), ws, ws_bytes, stream,
                       uses_ws);
+    // batch 1, mu = 8, per-row scales: the table precompute as its own kernel
+    // when asked for (and the workspace has room for the tables); otherwise,
+    // for large layers, the warp-specialised kernel (B200, batch 1:
+    // 28672x8192 25.3 -> 22.0 us, 8192x28672 29.1 -> 21.2 us; 11008x4096
+    // 8.0 -> 8.6 us and 4096x4096 5.4 -> 6.0 us, which stay on the kernel
+    // below).  With the precompute as its own kernel the same layers measured
+    // 25.2 and 31.3 us: the lookups alone took longer than the warp-specialised
+    // kernel with its in-CTA build, and the precompute ran before them.
+    if (B == 1 && mu == 8 && g.rgroup == 0 && (!nb1 || s->rgroup == 0)) {
+        const int64_t U = branch_units(g.ncols, g.nb, mu) + (nb1 ? branch_units(s->ncols, nb1, mu) : 0);
+        if (flags & kFlagSeparateTables) {
+            if (!ws || ws_bytes < workspace_bytes_for(M, 1) + table_bytes_for(U)) return FLUXBIN_ERR_WORKSPACE;
+            if (!aligned(ws, 16)) return FLUXBIN_ERR_MISALIGNED;
+            return run_lut1h(M, N, g, s, nb1, d_x, d_y, flags & ~kFlagSeparateTables, ws, stream, uses_ws);
+        }
+        if ((int64_t)M * N >= ((int64_t)1 << 27))
+            return run_lut1(M, N, g, s, nb1, d_x, d_y, flags, ws, ws_bytes, stream, uses_ws);
+    } else if (flags & kFlagSeparateTables) {
+        return FLUXBIN_ERR_UNSUPPORTED;
+    }
     // salient row scales finer than a unit: grouped visit order, one batch row per CTA
     const int gs1 = (nb1 && s->rgroup > 0 && s->rgroup < unit_cols(nb1, mu)) ? s->rgroup / mu : 0;
     const int bt = gs1 ? 1 : batch_tile(mu, B);
     KernelFn fn = mu == 8 ? select_kernel_mu8(g.nb, nb1, bt, gs1) : select_kernel_mu4(g.nb, nb1, bt, gs1);
     if (!fn) return FLUXBIN_ERR_UNSUPPORTED;
-
 
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return FLUXBIN_ERR_CUDA;
@@ -402,7 +664,7 @@ int run(int32_t M, int32_t N, int mu, const BranchIn& g, const BranchIn* s, cons
         st = func_info(fn, dev, mu, bt, gs1, di, &fi);
         if (st != FLUXBIN_OK) return st;
         const bool have_ws = ws && ws_bytes >= workspace_bytes_for(M, B) && aligned(ws, 16);
-        plan = make_plan(fn, dev, mu, bt, gs1, a.Ms, U, n_bc, di, fi, have_ws);
+        plan = make_plan(fn, dev, v1_shape(mu, bt, gs1), a.Ms, U, n_bc, di, fi, have_ws);
         // The build with three CTAs per SM (80 registers, a few bytes spilled)
         // pays where its extra slots widen the split: large layers (B200,
         // batch 1: 28672x8192 27.3 -> 25.8 us, 8192x28672 32.7 -> 29.5 us;
@@ -414,7 +676,7 @@ int run(int32_t M, int32_t N, int mu, const BranchIn& g, const BranchIn* s, cons
             KernelFn f3 = select_kernel_mu8_3(g.nb, nb1, bt, gs1);
             FuncInfo fi3;
             if (f3 && func_info(f3, dev, mu, bt, gs1, di, &fi3) == FLUXBIN_OK) {
-                const Plan p3 = make_plan(f3, dev, mu, bt, gs1, a.Ms, U, n_bc, di, fi3, have_ws);
+                const Plan p3 = make_plan(f3, dev, v1_shape(mu, bt, gs1), a.Ms, U, n_bc, di, fi3, have_ws);
                 const bool large = (int64_t)M * N >= ((int64_t)1 << 27);
                 if ((large && (B == 1 || p3.n_ks > plan.n_ks)) || (plan.n_ks == 1 && p3.n_ks >= 2)) {
                     fn = f3;
@@ -509,6 +771,17 @@ int fluxbin_device_status(uint32_t* out_flags) {
     if (e == cudaSuccess && v) e = cudaMemset(err, 0, sizeof(v));
     if (e != cudaSuccess) return cuda_fail(e);
     *out_flags = v;
+    return FLUXBIN_OK;
+}
+
+int fluxbin_layer_workspace_bytes(const fluxbin_layer_desc* desc, int32_t B, size_t* bytes) {
+    if (!bytes) return FLUXBIN_ERR_INVALID_ARG;
+    const int st = validate_desc(desc);
+    if (st != FLUXBIN_OK) return st;
+    if (B < 0) return FLUXBIN_ERR_BAD_SHAPE;
+    size_t n = workspace_bytes_for(desc->M, B);
+    if (desc->M > 0 && hoistable(*desc, B)) n += table_bytes_for(layer_units(*desc));
+    *bytes = n;
     return FLUXBIN_OK;
 }
 

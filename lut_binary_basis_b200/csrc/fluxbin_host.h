@@ -54,4 +54,18 @@ inline size_t workspace_bytes_for(int64_t M, int64_t B) {
     return acc + ((cnt + 255) & ~(size_t)255);
 }
 
+// Table buffer of the batch-1 path with the precompute as its own kernel:
+// one 64 KiB block per pair of units (fluxbin_tables.cuh).
+inline size_t table_bytes_for(int64_t units) { return units > 0 ? (size_t)((units + 1) / 2) * 65536u : 0u; }
+
+// Whether a layer at batch B can run its table precompute as a separate
+// kernel (batch 1, mu = 8, per-row scales in both branches).
+inline bool hoistable(const fluxbin_layer_desc& d, int64_t B) {
+    return B == 1 && d.mu == 8 && d.row_scale_group == 0 && (!has_salient(d) || d.sal_scale_group == 0);
+}
+
+inline int64_t layer_units(const fluxbin_layer_desc& d) {
+    return branch_units(d.N, d.Kb, d.mu) + (has_salient(d) ? branch_units(d.n_sal, d.Ks, d.mu) : 0);
+}
+
 }  // namespace fluxbin

@@ -80,6 +80,7 @@ struct KernelArgs {
     uint32_t flags;
     float* ws_acc;          // [B][Mp] split-K partial sums (zero between calls)
     unsigned int* ws_cnt;   // [n_rg * n_bc] arrival counters (zero between calls)
+    unsigned int* err;      // device error word (kernels with bounded waits set a bit when one gives up)
 };
 
 constexpr uint32_t kFlagAccumulate = 1u;
@@ -88,6 +89,7 @@ constexpr uint32_t kFlagEarlyWeights = 4u;
 constexpr uint32_t kFlagPathLut = 8u;
 constexpr uint32_t kFlagPathTc = 16u;
 constexpr uint32_t kFlagTestWaitTimeout = 32u;
+constexpr uint32_t kFlagSeparateTables = 64u;
 
 template <int MU, int BT>
 struct Geom {

@@ -1,0 +1,103 @@
+// FluxBin table precompute as a separate operator (sm_100a).
+//
+// The LUT Tensor Core notes (Section 3.1.1) move the table precompute out of
+// the lookup kernel into an operator of its own, run once and read by every
+// lookup unit, instead of rebuilding the same tables in every CTA that needs
+// them.  This kernel builds, for one layer and one activation row, every
+// unit's 32 tables of 2^8 signed partial sums of v = c (.) x (scale fusion,
+// FluxBin summary, Section 3 "LUT-Based GEMV Kernel"; the salient branch
+// gathers x and its column scales through its column map, Section 3 "Virtual
+// Columnar Mapping") into a global table buffer that the batch-1 lookup
+// kernel (fluxbin_lut1h.cuh) copies into shared memory with bulk copies.
+//
+// Table buffer layout (fp32): units are paired, v = u / 2, h = u % 2; entry e
+// of table (bank) b of unit u at byte
+//     v * 65536 + e * 256 + h * 128 + b * 4,
+// which is exactly the shared-memory layout the lookups address (one 64 KiB
+// copy per unit pair).  The bank of table (base k, sub-vector j) is k*P + j.
+//
+// One CTA of 256 threads builds one unit pair: the 512 activation products
+// (two per thread) go to shared memory, then thread t builds, for unit
+// 2v + t/128, the 16 entries of pattern block (t%128)/8 of the four tables in
+// banks 4*(t%8) .. 4*(t%8)+3 in Gray-code order (two paired fp32 adds and one
+// 16-byte store per step).
+#pragma once
+
+#include "fluxbin_kernel.cuh"
+
+namespace fluxbin {
+
+constexpr int kTabThreads = 256;
+constexpr int kTabPairBytes = 65536;
+
+__device__ __forceinline__ void stg_v4(float* p, uint64_t lo, uint64_t hi) {
+    asm volatile("st.global.v2.b64 [%0], {%1, %2};" ::"l"(p), "l"(lo), "l"(hi) : "memory");
+}
+
+template <int NB0, int NB1>
+__global__ void __launch_bounds__(kTabThreads) fluxbin_tables_kernel(const KernelArgs a, float* tables) {
+    __shared__ __align__(16) float vbuf[2][8][32];   // [unit of the pair][bit t][bank]
+    const int tid = threadIdx.x;
+    const int U = a.br[0].units + (NB1 > 0 ? a.br[1].units : 0);
+    const int v = blockIdx.x;
+    asm volatile("griddepcontrol.launch_dependents;");
+    // layer data of this thread's two product slots (before the dependency wait)
+    SlotRaw raw[2];
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+        const int u = 2 * v + q;
+        raw[q] = SlotRaw{__float2half(0.f), -1};
+        if (u < U) raw[q] = slot_raw<8, NB0, NB1>(a, u, tid);
+    }
+    // x was written by the preceding kernel; the table buffer may still be
+    // read by it
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+        const SlotStatic s = resolve_slot(a, raw[q]);
+        __half xv[1];
+        slot_x<1>(a, 0, s.col, xv);
+        vbuf[q][tid / 32][tid % 32] = s.c * __half2float(xv[0]);
+    }
+    __syncthreads();
+    const int q = tid / 128, it = tid % 128;
+    if (2 * v + q >= U) return;
+    const int hi = it / 8, qd = it % 8;
+    constexpr uint64_t kSign2 = 0x8000000080000000ull;
+    uint64_t T0 = 0, T1 = 0, d0[4], d1[4];
+#pragma unroll
+    for (int t = 4; t < 8; ++t) {
+        const uint64_t flip = ((hi >> (t - 4)) & 1) ? 0ull : kSign2;
+        const uint64_t v0 = *reinterpret_cast<const uint64_t*>(&vbuf[q][t][4 * qd]) ^ flip;
+        const uint64_t v1 = *reinterpret_cast<const uint64_t*>(&vbuf[q][t][4 * qd + 2]) ^ flip;
+        T0 = t == 4 ? v0 : add_f32x2(T0, v0);
+        T1 = t == 4 ? v1 : add_f32x2(T1, v1);
+    }
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+        const uint64_t v0 = *reinterpret_cast<const uint64_t*>(&vbuf[q][t][4 * qd]);
+        const uint64_t v1 = *reinterpret_cast<const uint64_t*>(&vbuf[q][t][4 * qd + 2]);
+        T0 = sub_f32x2(T0, v0);
+        T1 = sub_f32x2(T1, v1);
+        d0[t] = add_f32x2(v0, v0);
+        d1[t] = add_f32x2(v1, v1);
+    }
+    // entry e of bank 4 qd at float index v*16384 + e*64 + q*32 + 4 qd
+    float* base = tables + (int64_t)v * (kTabPairBytes / 4) + (hi << 4) * 64 + q * 32 + 4 * qd;
+    stg_v4(base, T0, T1);
+    static_for<1, 16>([&](auto ic) {
+        constexpr int i = decltype(ic)::value;
+        constexpr int t = lowest_bit(i);
+        constexpr int g = i ^ (i >> 1);
+        if constexpr ((g >> t) & 1) {
+            T0 = add_f32x2(T0, d0[t]);
+            T1 = add_f32x2(T1, d1[t]);
+        } else {
+            T0 = sub_f32x2(T0, d0[t]);
+            T1 = sub_f32x2(T1, d1[t]);
+        }
+        stg_v4(base + g * 64, T0, T1);
+    });
+}
+
+}  // namespace fluxbin

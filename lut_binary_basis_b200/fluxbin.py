@@ -23,6 +23,7 @@ FLAG_EARLY_WEIGHTS = 4
 FLAG_PATH_LUT = 8
 FLAG_PATH_TC = 16
 FLAG_TEST_WAIT_TIMEOUT = 32
+FLAG_SEPARATE_TABLES = 64
 
 STATUS = {0: "FLUXBIN_OK", -1: "FLUXBIN_ERR_INVALID_ARG", -2: "FLUXBIN_ERR_BAD_SHAPE",
           -3: "FLUXBIN_ERR_MISALIGNED", -4: "FLUXBIN_ERR_UNSUPPORTED", -5: "FLUXBIN_ERR_SMEM_BUDGET",
@@ -73,13 +74,15 @@ def lib():
             L.fluxbin_packed_sizes.argtypes = [P, ctypes.POINTER(sz), ctypes.POINTER(sz)]
             L.fluxbin_pack.argtypes = [P, P, P, P, P, P]
             L.fluxbin_workspace_bytes.argtypes = [i32, i32, ctypes.POINTER(sz)]
+            L.fluxbin_layer_workspace_bytes.argtypes = [P, i32, ctypes.POINTER(sz)]
             L.fluxbin_lut_gemv.argtypes = [i32, i32, i32, i32, i32, i32, P, P, P, P, P, i32, P, u32, P, sz, P]
             L.fluxbin_linear.argtypes = [P, P, P, P, P, P, P, P, P, i32, P, u32, P, sz, P]
             L.fluxbin_linear_static_scratch.argtypes = [P, P, P, P, P, P, P, P, P, i32, P, u32, P]
             L.fluxbin_device_status.argtypes = [ctypes.POINTER(u32)]
             L.fluxbin_fit.argtypes = [i32, i32, i32, i32, i32, P, P, P, P, P, P]
             L.fluxbin_fit_hybrid.argtypes = [i32, i32, i32, i32, i32, i32, P, i32, i32, P, P, P, P, P, P, P, P, P]
-            for f in ("fluxbin_packed_sizes", "fluxbin_pack", "fluxbin_workspace_bytes", "fluxbin_lut_gemv",
+            for f in ("fluxbin_packed_sizes", "fluxbin_pack", "fluxbin_workspace_bytes",
+                      "fluxbin_layer_workspace_bytes", "fluxbin_lut_gemv",
                       "fluxbin_linear", "fluxbin_linear_static_scratch", "fluxbin_device_status", "fluxbin_fit",
                       "fluxbin_fit_hybrid"):
                 getattr(L, f).restype = ctypes.c_int
@@ -139,6 +142,13 @@ def fluxbin_pack(desc: LayerDesc, signs: np.ndarray, sal_signs: Optional[np.ndar
 def fluxbin_workspace_bytes(M: int, B: int) -> int:
     n = ctypes.c_size_t()
     _check(lib().fluxbin_workspace_bytes(int(M), int(B), ctypes.byref(n)), "fluxbin_workspace_bytes")
+    return n.value
+
+
+def fluxbin_layer_workspace_bytes(desc: LayerDesc, B: int) -> int:
+    n = ctypes.c_size_t()
+    _check(lib().fluxbin_layer_workspace_bytes(ctypes.byref(desc), int(B), ctypes.byref(n)),
+           "fluxbin_layer_workspace_bytes")
     return n.value
 
 
@@ -273,6 +283,13 @@ class DeviceLayer:
         return cls(p["desc"], dev(p["words"], np.int32), dev(p["r"], np.float16), dev(p["c"], np.float16),
                    dev(p["swords"], np.int32), dev(p["rs"], np.float16), dev(p["cs"], np.float16),
                    dev(p["idx"], np.int32))
+
+    def workspace(self, B: int, device=None):
+        """A zero-filled workspace of fluxbin_layer_workspace_bytes(desc, B) bytes
+        (room for the batch-1 table buffer where the layer can use one)."""
+        import torch
+        n = max(fluxbin_layer_workspace_bytes(self.desc, B), 256)
+        return torch.zeros(n // 4, dtype=torch.int32, device=device if device is not None else self.words.device)
 
     def linear(self, x, y, flags: int = FLAG_Y_FP32, workspace=None, stream=None) -> None:
         B = x.shape[0] if x.dim() == 2 else 1

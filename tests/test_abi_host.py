@@ -134,7 +134,8 @@ def test_device_entry_points_validate_before_any_cuda_call():
     assert _linear_status(desc, y=0) == -1
     assert _linear_status(desc, y=0x1002) == -3      # fp32 y needs 4-byte alignment
     assert _linear_status(desc, words=0x1008) == -3  # packed words need 16-byte alignment
-    assert _linear_status(desc, flags=64) == -1
+    assert _linear_status(desc, flags=128) == -1      # unknown flag
+    assert _linear_status(desc, flags=fluxbin.FLAG_Y_FP32 | fluxbin.FLAG_SEPARATE_TABLES) == -6  # no table buffer
     assert _linear_status(LayerDesc(32, 64, 2, 1, 4, 6, 0, 0)) == -4
     L = fluxbin.lib()
     assert L.fluxbin_lut_gemv(32, 64, 65, 2, 8, 0, 0x1000, 0x2000, 0x3000, None, 0x4000, 1, 0x5000,
@@ -142,3 +143,18 @@ def test_device_entry_points_validate_before_any_cuda_call():
     assert L.fluxbin_lut_gemv(32, 64, 64, 3, 8, 0, 0x1000, 0x2000, 0x3000, None, 0x4000, 1, 0x5000,
                               fluxbin.FLAG_Y_FP32, None, 0, None) == -4
     assert L.fluxbin_linear(None, 0, 0, 0, 0, 0, 0, 0, 0, 1, 0, 0, None, 0, None) == -1
+
+
+def test_layer_workspace_bytes():
+    """Batch-1 mu = 8 layers with per-row scales add a table buffer of 64 KiB
+    per pair of units (a unit is (32/nb)*mu columns of a branch); other layers
+    and batch sizes need exactly fluxbin_workspace_bytes."""
+    d = LayerDesc(28672, 8192, 2, 2, 246, 8, 0, 0)
+    units = -(-8192 // 128) + -(-246 // 128)
+    assert fluxbin.fluxbin_layer_workspace_bytes(d, 1) == \
+        fluxbin.fluxbin_workspace_bytes(28672, 1) + -(-units // 2) * 65536
+    for desc, B in ((d, 2), (LayerDesc(4096, 4096, 2, 1, 205, 4, 0, 0), 1),
+                    (LayerDesc(4096, 4096, 2, 2, 512, 8, 128, 16), 1)):
+        assert fluxbin.fluxbin_layer_workspace_bytes(desc, B) == fluxbin.fluxbin_workspace_bytes(desc.M, B)
+    with pytest.raises(fluxbin.FluxbinError):
+        fluxbin.fluxbin_layer_workspace_bytes(LayerDesc(4, 4, 3, 0, 0, 8, 0, 0), 1)

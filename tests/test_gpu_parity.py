@@ -187,14 +187,22 @@ def test_noop_and_errors_on_device():
     x = torch.zeros((0, sp.N), dtype=torch.float16, device="cuda")
     y = torch.zeros((0, sp.M), dtype=torch.float32, device="cuda")
     d.linear(x, y, fluxbin.FLAG_Y_FP32, None)   # B = 0: nothing to do
-    # a layer whose reduction is split wider than a cluster refuses to run
-    # without a workspace (few rows, very long rows)
+    # a layer that would split its long rows through a workspace runs on
+    # thread-block clusters (or unsplit) when the caller gives none
     big = spec(256, 65536, 2, 1, 205, 8)
-    lb = fluxbin.DeviceLayer.from_host(synth.make_layer(big, [97]))
-    xb = torch.zeros((1, big.N), dtype=torch.float16, device="cuda")
-    yb = torch.zeros((1, big.M), dtype=torch.float32, device="cuda")
+    hl = synth.make_layer(big, [97])
+    lb = fluxbin.DeviceLayer.from_host(hl)
+    for B in (1, 2):
+        xh = synth.make_x(big, B, [98, B])
+        yb = torch.full((B, big.M), float("nan"), dtype=torch.float32, device="cuda")
+        lb.linear(torch.from_numpy(xh).cuda(), yb, fluxbin.FLAG_Y_FP32, None)
+        torch.cuda.synchronize()
+        assert_close(yb.cpu().numpy().astype(np.float64), oracle.linear(hl, xh), hl, xh)
+    # the tensor-core path always needs one
+    xb = torch.zeros((16, big.N), dtype=torch.float16, device="cuda")
+    yb = torch.zeros((16, big.M), dtype=torch.float32, device="cuda")
     with pytest.raises(fluxbin.FluxbinError) as e:
-        lb.linear(xb, yb, fluxbin.FLAG_Y_FP32, None)
+        lb.linear(xb, yb, fluxbin.FLAG_Y_FP32 | fluxbin.FLAG_PATH_TC, None)
     assert e.value.status == -6
 
 
