@@ -52,7 +52,11 @@ def _load():
                                                i32, P, i64, P, P]
             lib.oracle_linear_rows.restype = None
             lib.oracle_lut_linear_rows.argtypes = [i64, i64, i32, i32, P, P, P, i32, i64, i32, P, P, P, P,
-                                                   i32, i32, i32, P, i64, P, P]
+                                                   i32, i32, i32, i32, P, i64, P, P]
+            lib.oracle_round_fp16.argtypes = [ctypes.c_double]
+            lib.oracle_round_fp16.restype = ctypes.c_double
+            lib.oracle_quantize_table_int8.argtypes = [P, i64]
+            lib.oracle_quantize_table_int8.restype = ctypes.c_double
             lib.oracle_lut_linear_rows.restype = i32
             lib.oracle_lut_table.argtypes = [P, i32, P]
             lib.oracle_lut_table_sym.argtypes = [P, i32, P]
@@ -152,10 +156,27 @@ def gemv_rows(W: np.ndarray, x) -> np.ndarray:
     return y
 
 
-def lut_linear(layer, x, mu: int, sym: bool = False, rows: Optional[Sequence[int]] = None) -> np.ndarray:
+TABLE_QUANT = {"none": 0, "fp16": 1, "int8": 2}
+
+
+def round_fp16(v: float) -> float:
+    """The binary16 value nearest to v (ties to even)."""
+    return float(_load().oracle_round_fp16(float(v)))
+
+
+def quantize_table_int8(T) -> tuple:
+    """INT8 quantisation of one table with one scale: returns (entries, scale)."""
+    tt = _f64(T).copy()
+    s = float(_load().oracle_quantize_table_int8(_ptr(tt), tt.size))
+    return tt, s
+
+
+def lut_linear(layer, x, mu: int, sym: bool = False, rows: Optional[Sequence[int]] = None,
+               tables: str = "none") -> np.ndarray:
     """The same layer evaluated by the method's steps: scale-fused tables of
     2^mu signed partial sums per sub-vector, looked up by the sign patterns
-    (``sym``: symmetric half tables)."""
+    (``sym``: symmetric half tables; ``tables``: table quantisation, "none",
+    "fp16" or "int8" with one scale per table)."""
     L = _unpack(layer)
     xx = _f64(x)
     B = xx.shape[0]
@@ -166,7 +187,7 @@ def lut_linear(layer, x, mu: int, sym: bool = False, rows: Optional[Sequence[int
     rc = _load().oracle_lut_linear_rows(L["M"], L["N"], L["Kb"], L["G"], _ptr(L["signs"]), _ptr(L["r"]),
                                         _ptr(L["c"]), L["Ks"], L["n_sal"], L["Gs"], _ptr(L["sal_signs"]),
                                         _ptr(L["rs"]), _ptr(L["cs"]), _ptr(L["sal_idx"]), int(mu), int(bool(sym)),
-                                        B, _ptr(xx), rr.size, _ptr(rr), _ptr(y))
+                                        TABLE_QUANT[tables], B, _ptr(xx), rr.size, _ptr(rr), _ptr(y))
     if rc != 0:
         raise ValueError("scale block sizes must be multiples of mu")
     return y

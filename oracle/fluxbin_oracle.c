@@ -33,6 +33,7 @@
  *   bit value 1 means +1, 0 means -1; bit t of a pattern is column j*mu + t;
  *   the symmetric half table keeps the entries whose top bit (t = mu-1) is 0.
  */
+#include <math.h>
 #include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
@@ -176,6 +177,60 @@ double oracle_lut_lookup_sym(const double* Th, int mu, int64_t p) {
 }
 
 /*
+ * Table quantisation (LUT Tensor Core notes, Section 3.1.3: the precomputed
+ * table entries are stored in a lower precision than the activations).
+ *
+ * oracle_round_fp16: the IEEE binary16 value nearest to v (ties to the even
+ * significand), from the format's definition: 10 fraction bits, exponents
+ * -14 .. 15, subnormal spacing 2^-24, values at or beyond 65520 overflow.
+ */
+double oracle_round_fp16(double v) {
+    if (v != v) return v;
+    double a = fabs(v);
+    if (a >= 65520.0) return v > 0 ? INFINITY : -INFINITY;
+    int e;
+    (void)frexp(a, &e);                   /* a = f * 2^e, 0.5 <= f < 1 */
+    int ex = e - 1;                       /* a in [2^ex, 2^(ex+1)) */
+    if (ex < -14) ex = -14;               /* subnormals share the spacing of the smallest binade */
+    double ulp = ldexp(1.0, ex - 10);
+    double q = a / ulp;                   /* exact: a power-of-two scaling */
+    double r = floor(q);
+    double frac = q - r;
+    if (frac > 0.5 || (frac == 0.5 && fmod(r, 2.0) != 0.0)) r += 1.0;
+    return copysign(r * ulp, v);
+}
+
+/*
+ * INT8 table with one scale per table: s = max_p |T[p]| / 127 and every
+ * entry replaced by s * q, q the integer nearest to T[p] / s (ties to even),
+ * |q| <= 127.  An all-zero table stays zero.  Returns s.
+ */
+double oracle_quantize_table_int8(double* T, int64_t E) {
+    double m = 0.0;
+    for (int64_t p = 0; p < E; ++p)
+        if (fabs(T[p]) > m) m = fabs(T[p]);
+    if (m == 0.0) return 0.0;
+    double s = m / 127.0;
+    for (int64_t p = 0; p < E; ++p) {
+        double q = T[p] / s, r = floor(q), frac = q - r;
+        if (frac > 0.5 || (frac == 0.5 && fmod(r, 2.0) != 0.0)) r += 1.0;
+        if (r > 127.0) r = 127.0;
+        if (r < -127.0) r = -127.0;
+        T[p] = r * s;
+    }
+    return s;
+}
+
+/* Applies table quantisation mode tq (0: none, 1: fp16 entries, 2: INT8 per table). */
+static void quantize_table(double* T, int64_t E, int tq) {
+    if (tq == 1) {
+        for (int64_t p = 0; p < E; ++p) T[p] = oracle_round_fp16(T[p]);
+    } else if (tq == 2) {
+        (void)oracle_quantize_table_int8(T, E);
+    }
+}
+
+/*
  * One branch in LUT form, for every requested row:
  *   acc_k,g(i) = sum over sub-vectors j of the block g of T_{k,j}[pattern of B_k[i][j*mu .. j*mu+mu-1]]
  *   y(i)      += sum_{k,g} r_k(i, g) acc_k,g(i)
@@ -186,7 +241,7 @@ double oracle_lut_lookup_sym(const double* Th, int mu, int64_t p) {
 static void lut_branch_rows(int64_t M, int64_t ncols, int64_t N, int nb, int mu, int G,
                             const int8_t* signs, const double* r, const double* c,
                             const int32_t* gather, int B, const double* x,
-                            int64_t nrows, const int64_t* rows, int sym, double* y) {
+                            int64_t nrows, const int64_t* rows, int sym, int tq, double* y) {
     int64_t nsub = (ncols + mu - 1) / mu;
     int64_t E = (int64_t)1 << mu;
     int64_t Estore = sym ? (E >> 1) : E;
@@ -203,6 +258,7 @@ static void lut_branch_rows(int64_t M, int64_t ncols, int64_t N, int nb, int mu,
                 }
                 double* T = tab + ((int64_t)k * nsub + j) * Estore;
                 if (sym) oracle_lut_table_sym(v, mu, T); else oracle_lut_table(v, mu, T);
+                quantize_table(T, Estore, tq);
             }
         /* Lookup and accumulate; the row scale multiplies the accumulated sum. */
         for (int64_t q = 0; q < nrows; ++q) {
@@ -247,7 +303,8 @@ static void lut_branch_rows(int64_t M, int64_t ncols, int64_t N, int nb, int mu,
  * The full layer in LUT form: the global branch over the N input columns,
  * plus the salient branch over its dense n_sal columns whose activations and
  * scales are gathered through sal_idx (Virtual Columnar Mapping).
- * sym != 0 uses the symmetric half tables.  Signs must be +-1 here (a zero
+ * sym != 0 uses the symmetric half tables; tq quantises every table after it
+ * is built (0: none, 1: fp16 entries, 2: INT8 with a per-table scale).  Signs must be +-1 here (a zero
  * has no bit pattern).  Block sizes G and Gs must be multiples of mu.
  * Returns 0, or -1 if a block size does not hold whole sub-vectors.
  */
@@ -255,13 +312,13 @@ int oracle_lut_linear_rows(int64_t M, int64_t N, int Kb, int G,
                            const int8_t* signs, const double* r, const double* c,
                            int Ks, int64_t n_sal, int Gs,
                            const int8_t* sal_signs, const double* rs, const double* cs,
-                           const int32_t* sal_idx, int mu, int sym,
+                           const int32_t* sal_idx, int mu, int sym, int tq,
                            int B, const double* x,
                            int64_t nrows, const int64_t* rows, double* y) {
-    if ((G > 0 && G % mu) || (Gs > 0 && Gs % mu) || mu < 1 || mu > 16) return -1;
+    if ((G > 0 && G % mu) || (Gs > 0 && Gs % mu) || mu < 1 || mu > 16 || tq < 0 || tq > 2) return -1;
     memset(y, 0, sizeof(double) * (size_t)(B * nrows));
-    lut_branch_rows(M, N, N, Kb, mu, G, signs, r, c, NULL, B, x, nrows, rows, sym, y);
+    lut_branch_rows(M, N, N, Kb, mu, G, signs, r, c, NULL, B, x, nrows, rows, sym, tq, y);
     if (Ks > 0 && n_sal > 0)
-        lut_branch_rows(M, n_sal, N, Ks, mu, Gs, sal_signs, rs, cs, sal_idx, B, x, nrows, rows, sym, y);
+        lut_branch_rows(M, n_sal, N, Ks, mu, Gs, sal_signs, rs, cs, sal_idx, B, x, nrows, rows, sym, tq, y);
     return 0;
 }
