@@ -154,16 +154,22 @@ typedef struct fluxbin_layer_desc {
  * Two execution paths compute the same layer.  The LUT path builds the 2^mu
  * signed partial sums of every activation sub-vector in shared memory and
  * looks them up with the packed bit patterns (FluxBin summary, Section 3
- * "LUT-Based GEMV Kernel").  The tensor-core path, for larger batches, expands
- * the +-1 signs of each unit into fp16 in shared memory only and contracts them
- * with the fp16 products c (.) x on the tensor cores (tcgen05.mma), fp32
- * accumulation in tensor memory, row scales applied to the accumulators (the
- * LUT Tensor Core notes, Section 2.2, read LUT-based mixed-precision GEMM as a
- * GEMM with one low-bit operand).  It needs mu == 4 or 8, per-row scales
- * (row_scale_group == 0 and sal_scale_group == 0) and a workspace; it is taken
- * by default for a qualifying layer when B >= 16 and M * N > 4096 * 4096, or
- * when B >= 8 and M >= 16384 (where it measured faster on B200), and may be
- * forced either way with the flags above.  Its products are rounded to fp16 before the
+ * "LUT-Based GEMV Kernel").  At mu = 8 with per-row scales and a batch of 2 or
+ * more (batch 2 only above 4096 x 4096), the LUT path keeps the tables of two
+ * batch rows in one fp16 pair per entry (table quantisation to fp16, LUT Tensor
+ * Core notes, Section 3.1.3): one lookup serves both rows; the entries are
+ * rounded to fp16 once and the entries of two consecutive steps are added in
+ * fp16 before the fp32 accumulation (relative error of y about 3e-4 on the
+ * benchmark layers).  The tensor-core path expands the +-1 signs of each unit
+ * into fp16 in shared memory only and contracts them with the fp16 products
+ * c (.) x on the tensor cores (tcgen05.mma), fp32 accumulation in tensor
+ * memory, row scales applied to the accumulators (the LUT Tensor Core notes,
+ * Section 2.2, read LUT-based mixed-precision GEMM as a GEMM with one low-bit
+ * operand).  It needs mu == 4 or 8, per-row scales (row_scale_group == 0 and
+ * sal_scale_group == 0) and a workspace; it is taken by default only for
+ * mu = 4 layers with B >= 16 and M * N > 4096 * 4096, or B >= 8 and
+ * M >= 16384 (where it measured faster on B200), and may be forced either way
+ * with the flags above.  Its products are rounded to fp16 before the
  * contraction (relative error below 2^-11 per product).
  */
 

@@ -25,6 +25,10 @@ KernelFn select_kernel_mu8_3(int nb0, int nb1, int bt, int gs1);
 using TcKernelFn = void (*)(TcArgs);
 TcKernelFn select_tc_kernel(int mu, int nb0, int nb1);
 KernelFn select_kernel_lut1(int lw, int nb0, int nb1);
+KernelFn select_kernel_lut2(int nb0, int nb1);
+int lut2_threads();
+int lut2_smem_bytes();
+int lut2_slabs();
 using TabKernelFn = void (*)(KernelArgs, float*);
 using HKernelFn = void (*)(KernelArgs, const float*);
 TabKernelFn select_tables_kernel(int nb0, int nb1);
@@ -36,13 +40,16 @@ int lut1_threads(int lw);
 int lut1_smem_bytes(int lw);
 int lut1_slabs(int lw);
 
-// Automatic path choice for a layer both paths can run.  Measured on B200
-// (µs per call, LUT / tensor cores): 4096x4096 B=8 17.6/35.7, B=16 31.0/38.1;
-// 4096x11008 B=8 40.4/60.4, B=16 76.3/65.0; 11008x4096 B=8 58.9/58.7,
-// B=16 112.5/63.0; 28672x8192 B=8 244/183, B=16 451/196; 8192x28672 (mu=4)
-// B=8 241/255, B=16 473/256.  The tensor cores win from batch 16 on layers
-// above 4096x4096 and from batch 8 on layers with at least 16384 rows.
-static bool prefer_tensor_cores(int64_t M, int64_t N, int B) {
+// Automatic path choice for a layer both paths can run.  At mu = 8 the LUT
+// path on fp16-pair tables (fluxbin_lut2.cuh) is faster than the tensor cores
+// at every batch measured on B200 (us per call, LUT / tensor cores):
+// 28672x8192 B=8 91.5/183, B=16 182/196; 8192x28672 B=16 161/208;
+// 11008x4096 B=16 46.5/64.0; 4096x11008 B=16 34.0/65.9.  At mu = 4 (tables
+// of one row, fluxbin_kernel.cuh): 4096x4096 B=16 31.0/38.1; 8192x28672 B=8
+// 241/255, B=16 473/256; the tensor cores win from batch 16 on layers above
+// 4096x4096 and from batch 8 on layers with at least 16384 rows.
+static bool prefer_tensor_cores(int64_t M, int64_t N, int B, int mu) {
+    if (mu == 8) return false;
     return (B >= 16 && M * N > (int64_t)4096 * 4096) || (B >= 8 && M >= 16384);
 }
 
@@ -476,6 +483,82 @@ int run_lut1(int32_t M, int32_t N, const BranchIn& g, const BranchIn* s, int nb1
     return FLUXBIN_OK;
 }
 
+// Batches of 2-16, mu = 8, per-row scales: pairs of batch rows on fp16-pair
+// tables (fluxbin_lut2.cuh), one CTA per SM, 1024 rows x one batch pair x a
+// range of units per CTA.
+int run_lut2(int32_t M, int32_t N, const BranchIn& g, const BranchIn* s, int nb1, const uint16_t* d_x, int32_t B,
+             void* d_y, uint32_t flags, void* ws, size_t ws_bytes, void* stream, int* uses_ws) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return FLUXBIN_ERR_CUDA;
+    KernelArgs a = {};
+    fill_branches(a, 8, g, s, nb1);
+    a.Ms = (int32_t)row_slabs(M);
+    const int64_t U = (int64_t)a.br[0].units + a.br[1].units;
+    const int n_bp = (B + 1) / 2;
+    const bool have_ws = ws && ws_bytes >= workspace_bytes_for(M, B) && aligned(ws, 16);
+    DeviceInfo di;
+    unsigned int* err = nullptr;
+    KernelFn fn = select_kernel_lut2(g.nb, nb1);
+    if (!fn) return FLUXBIN_ERR_UNSUPPORTED;
+    Plan plan;
+    {
+        std::lock_guard<std::mutex> lock(g_mu);
+        int st = device_info(dev, &di);
+        if (st != FLUXBIN_OK) return st;
+        FuncInfo fi;
+        const CtaShape cs{lut2_slabs(), lut2_threads(), (size_t)lut2_smem_bytes()};
+        if ((st = func_info_shape(fn, dev, cs.smem, cs.threads, di, &fi)) != FLUXBIN_OK) return st;
+        plan = make_plan(fn, dev, cs, a.Ms, U, n_bp, di, fi, have_ws, true);
+    }
+    {
+        std::lock_guard<std::mutex> lock(g_tc_mu);
+        const int st = device_error_address(dev, &err);
+        if (st != FLUXBIN_OK) return st;
+    }
+    a.x = reinterpret_cast<const __half*>(d_x);
+    a.y = d_y;
+    a.M = M;
+    a.N = N;
+    a.B = B;
+    a.Mp = a.Ms * kLanes;
+    a.n_rg = plan.n_rg;
+    a.n_bc = n_bp;
+    a.n_ks = plan.n_ks;
+    a.cluster = plan.cluster ? 1 : 0;
+    a.flags = flags;
+    a.err = err;
+    if (uses_ws) {  // plan query only
+        *uses_ws = (a.n_ks > 1 && !plan.cluster) ? 1 : 0;
+        return FLUXBIN_OK;
+    }
+    if (a.n_ks > 1 && !plan.cluster) {
+        if (!have_ws) return FLUXBIN_ERR_WORKSPACE;
+        const size_t acc = (((size_t)B * a.Mp * sizeof(float)) + 255) & ~(size_t)255;
+        a.ws_acc = static_cast<float*>(ws);
+        a.ws_cnt = reinterpret_cast<unsigned int*>(static_cast<char*>(ws) + acc);
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)((int64_t)a.n_rg * a.n_bc * a.n_ks));
+    cfg.blockDim = dim3((unsigned)lut2_threads());
+    cfg.dynamicSmemBytes = (size_t)lut2_smem_bytes();
+    cfg.stream = static_cast<cudaStream_t>(stream);
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (plan.cluster) {
+        attr[1].id = cudaLaunchAttributeClusterDimension;
+        attr[1].val.clusterDim.x = (unsigned)a.n_ks;
+        attr[1].val.clusterDim.y = 1;
+        attr[1].val.clusterDim.z = 1;
+        cfg.numAttrs = 2;
+    }
+    const cudaError_t le = cudaLaunchKernelEx(&cfg, fn, a);
+    if (le != cudaSuccess) return cuda_fail(le);
+    return FLUXBIN_OK;
+}
+
 // Batch 1, mu = 8, per-row scales, with room for the table buffer in the
 // workspace: the table precompute as its own kernel (fluxbin_tables.cuh),
 // then the lookups on the precomputed tables (fluxbin_lut1h.cuh).  2048 rows
@@ -605,7 +688,7 @@ int run(int32_t M, int32_t N, int mu, const BranchIn& g, const BranchIn* s, cons
     const bool tc_fits = (mu == 8 || mu == 4) && g.rgroup == 0 && (!nb1 || s->rgroup == 0);
     if ((flags & kFlagPathTc) && !tc_fits) return FLUXBIN_ERR_UNSUPPORTED;
     if ((flags & kFlagPathTc) ||
-        (!(flags & (kFlagPathLut | kFlagSeparateTables)) && tc_fits && prefer_tensor_cores(M, N, B) && ws &&
+        (!(flags & (kFlagPathLut | kFlagSeparateTables)) && tc_fits && prefer_tensor_cores(M, N, B, mu) && ws &&
          ws_bytes >= workspace_bytes_for(M, B)))
         return run_tc(M, N, mu, g, s, nb1, d_x, B, d_y, flags & ~(kFlagPathLut | kFlagPathTc), ws, ws_bytes, stream,
                       uses_ws);
@@ -629,6 +712,14 @@ int run(int32_t M, int32_t N, int mu, const BranchIn& g, const BranchIn* s, cons
     } else if (flags & kFlagSeparateTables) {
         return FLUXBIN_ERR_UNSUPPORTED;
     }
+    // batches of 2-16, mu = 8, per-row scales: pairs of batch rows on
+    // fp16-pair tables (B200, us per call against one-row fp32 tables below:
+    // 28672x8192 B=2 26.4/49.0, B=4 47.0/104, B=16 182/346; 11008x4096 B=2
+    // 10.8/11.4, B=8 17.9/37.3; 4096x4096 B=4 8.9/9.4, B=16 15.0/26.7; only
+    // 4096x4096 at B=2 stays faster below, 6.5/7.1)
+    if (B >= 2 && mu == 8 && g.rgroup == 0 && (!nb1 || s->rgroup == 0) &&
+        (B >= 4 || (int64_t)M * N > (int64_t)4096 * 4096))
+        return run_lut2(M, N, g, s, nb1, d_x, B, d_y, flags, ws, ws_bytes, stream, uses_ws);
     // salient row scales finer than a unit: grouped visit order, one batch row per CTA
     const int gs1 = (nb1 && s->rgroup > 0 && s->rgroup < unit_cols(nb1, mu)) ? s->rgroup / mu : 0;
     const int bt = gs1 ? 1 : batch_tile(mu, B);

@@ -211,7 +211,8 @@ def test_noop_and_errors_on_device():
 # oracle runs over rows in parallel on the host cores), in the launch
 # configuration the benchmark times (packed words requested early, a caller
 # workspace).  Each (layer, batch) runs on the path the library chooses; the
-# batch-16 cases of the 70B-shaped layers also run forced onto the other path.
+# batch-16 cases of the 70B-shaped layers also run forced onto the other path
+# (tensor cores for mu = 8, the LUT path for mu = 4).
 # ---------------------------------------------------------------------------
 
 A, L, T = 0, fluxbin.FLAG_PATH_LUT, fluxbin.FLAG_PATH_TC
@@ -221,7 +222,7 @@ FULL = [
     (synth.layer_7b_proj(), 1, [(1, A)]),
     (synth.layers_7b_mlp()[0], 2, [(1, A), (2, A), (4, A), (8, A)]),
     (synth.layers_7b_mlp()[1], 2, [(1, A), (2, A), (4, A), (8, A)]),  # B = 1: split through the workspace
-    (synth.layers_70b_mlp(8)[0], 3, [(1, A), (16, A), (16, L)]),      # B = 1: three CTAs per SM
+    (synth.layers_70b_mlp(8)[0], 3, [(1, A), (2, A), (16, A), (16, T)]),   # B >= 2: fp16-pair tables
     (synth.layers_70b_mlp(8)[1], 3, [(1, A), (16, A)]),
     (synth.layers_70b_mlp(4)[0], 3, [(1, A), (16, A), (16, L)]),
     (synth.layers_70b_mlp(4)[1], 3, [(1, A), (16, A)]),
