@@ -166,6 +166,27 @@ __device__ __forceinline__ float table_entry(uint32_t byte_off) {
     return *reinterpret_cast<const float*>(fb_smem + OFF + byte_off);
 }
 
+// The dynamic shared memory of a kernel without static shared variables
+// starts right after the 1 KiB the system reserves per CTA (in a cluster
+// launch the CTA's rank sits in bits 24 and up of its shared addresses).
+// Kernels that address tables absolutely check this at entry and otherwise
+// take their add-based loop.
+constexpr uint32_t kDynSmemBase = 0x400u;
+
+// Table entry / entry word at an absolute shared address (+ a constant).
+template <int IMM>
+__device__ __forceinline__ float lds_f32_abs(uint32_t addr) {
+    float v;
+    asm volatile("ld.shared.f32 %0, [%1+%2];" : "=f"(v) : "r"(addr), "n"(IMM));
+    return v;
+}
+template <int IMM>
+__device__ __forceinline__ uint32_t lds_u32_abs(uint32_t addr) {
+    uint32_t v;
+    asm volatile("ld.shared.b32 %0, [%1+%2];" : "=r"(v) : "r"(addr), "n"(IMM));
+    return v;
+}
+
 // Shared-memory access by 32-bit shared address (+ a constant byte offset).
 __device__ __forceinline__ uint64_t lds_b64(uint32_t addr) {
     uint64_t v;
@@ -236,6 +257,20 @@ struct Offsets {
     __device__ __forceinline__ void load(int lane) {
 #pragma unroll
         for (int r = 0; r < 11; ++r) o[r] = __ldg(&kOffsetTable.w[nb_index<NB>()][order_index<GSV>()][r][lane]);
+    }
+    // Absolute addressing (mu = 8): with the CTA's rank byte in byte 3 of every
+    // offset word, (rank << 24) | (pattern << 8) | bank*4, byte 2 zero (the
+    // sign of a bank offset byte, below 128, replicated by the permute's
+    // sign mode); the shared base goes into the load's immediate.
+    __device__ __forceinline__ void set_rank_byte(uint32_t hi_byte) {
+#pragma unroll
+        for (int r = 0; r < 11; ++r) o[r] = (o[r] & 0x00FFFFFFu) | hi_byte;
+    }
+    __device__ __forceinline__ uint32_t addr_abs(uint32_t w, int q) const {
+        uint32_t d;
+        asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(w), "r"(o[q / 3]),
+            "r"((uint32_t)((4 + q % 3) | ((q % 4) << 4) | (0xC << 8) | (0x7 << 12))));
+        return d;
     }
     // table byte offset of the entry step q selects: (pattern << 8) | bank*4
     __device__ __forceinline__ uint32_t addr(uint32_t w, int q) const {

@@ -141,20 +141,27 @@ __device__ __forceinline__ void l2_build_unit(uint32_t sbase, int bt) {
     }
 }
 
-// 32 lookup steps of one lane for one row slab and unit (stage H), both rows.
-template <int NB, int H>
+// 32 lookup steps of one lane for one row slab and unit (stage H), both rows
+// (ABS: absolute addressing as in the batch-1 kernel).
+template <int NB, int H, bool ABS>
 __device__ __forceinline__ void l2_lookup_unit(const uint4 (&w)[2], const Offsets<8>& off, float (&acc)[NB][2]) {
     constexpr int P = 32 / NB;
 #pragma unroll
     for (int q = 0; q < 32; q += 2) {
-        const uint32_t a0 = off.addr(word_of(w[q / 16], (q / 4) % 4), q);
-        const uint32_t a1 = off.addr(word_of(w[(q + 1) / 16], ((q + 1) / 4) % 4), q + 1);
-        const uint32_t s = add_f16x2(table_word<H * 128>(a0), table_word<H * 128>(a1));
-        acc_f16x2(s, acc[q / P][0], acc[q / P][1]);
+        const uint32_t w0 = word_of(w[q / 16], (q / 4) % 4), w1 = word_of(w[(q + 1) / 16], ((q + 1) / 4) % 4);
+        uint32_t e0, e1;
+        if constexpr (ABS) {
+            e0 = lds_u32_abs<kDynSmemBase + H * 128>(off.addr_abs(w0, q));
+            e1 = lds_u32_abs<kDynSmemBase + H * 128>(off.addr_abs(w1, q + 1));
+        } else {
+            e0 = table_word<H * 128>(off.addr(w0, q));
+            e1 = table_word<H * 128>(off.addr(w1, q + 1));
+        }
+        acc_f16x2(add_f16x2(e0, e1), acc[q / P][0], acc[q / P][1]);
     }
 }
 
-template <int BR, int NB, int H>
+template <int BR, int NB, int H, bool ABS>
 __device__ __forceinline__ void l2_lookup_step(const KernelArgs& a, int u, int u_end, int k, int slab0, int lane,
                                                uint32_t full_bar, uint32_t empty_bar, const Offsets<8>& off,
                                                uint4 (&wr)[2][kSlabsPerWarp][2], float (&acc)[kSlabsPerWarp][NB][2],
@@ -162,7 +169,7 @@ __device__ __forceinline__ void l2_lookup_step(const KernelArgs& a, int u, int u
     if (ok) ok = l1_mbar_wait(full_bar, (uint32_t)((k >> 1) & 1));
 #pragma unroll
     for (int rs = 0; rs < kSlabsPerWarp; ++rs) {
-        l2_lookup_unit<NB, H>(wr[H][rs], off, acc[rs]);
+        l2_lookup_unit<NB, H, ABS>(wr[H][rs], off, acc[rs]);
         if (u + 2 < u_end) load_unit_slab<8, 1>(a, u + 2, slab0 + rs, lane, wr[H][rs]);
     }
     __syncwarp();
@@ -231,26 +238,37 @@ __global__ void __launch_bounds__(L2Geom<LW>::kThreads, 1) fluxbin_lut2_kernel(c
 #pragma unroll
                 for (int q = 0; q < NB1E; ++q) acc1[rs][q][r] = 0.f;
             }
-        int k = 0;
-        for (int u = u_begin; u < min(u_end, U0); ++u, ++k) {
-            if (k & 1)
-                l2_lookup_step<0, NB0, 1>(a, u, u_end, k, slab0, lane, full0 + 8, empty0 + 8, off, wr, acc0, ok);
-            else
-                l2_lookup_step<0, NB0, 0>(a, u, u_end, k, slab0, lane, full0, empty0, off, wr, acc0, ok);
-        }
-        if constexpr (NB1 > 0) {
-            if (max(u_begin, U0) < u_end) {
-                Offsets<8> off1;
-                off1.template load<NB1, 0>(lane);
-                for (int u = max(u_begin, U0); u < u_end; ++u, ++k) {
-                    if (k & 1)
-                        l2_lookup_step<1, NB1, 1>(a, u, u_end, k, slab0, lane, full0 + 8, empty0 + 8, off1, wr, acc1,
-                                                  ok);
-                    else
-                        l2_lookup_step<1, NB1, 0>(a, u, u_end, k, slab0, lane, full0, empty0, off1, wr, acc1, ok);
+        auto lookups = [&](auto abs_c) {
+            constexpr bool ABS = decltype(abs_c)::value;
+            if constexpr (ABS) off.set_rank_byte(sbase & 0xFF000000u);
+            int k = 0;
+            for (int u = u_begin; u < min(u_end, U0); ++u, ++k) {
+                if (k & 1)
+                    l2_lookup_step<0, NB0, 1, ABS>(a, u, u_end, k, slab0, lane, full0 + 8, empty0 + 8, off, wr, acc0,
+                                                   ok);
+                else
+                    l2_lookup_step<0, NB0, 0, ABS>(a, u, u_end, k, slab0, lane, full0, empty0, off, wr, acc0, ok);
+            }
+            if constexpr (NB1 > 0) {
+                if (max(u_begin, U0) < u_end) {
+                    Offsets<8> off1;
+                    off1.template load<NB1, 0>(lane);
+                    if constexpr (ABS) off1.set_rank_byte(sbase & 0xFF000000u);
+                    for (int u = max(u_begin, U0); u < u_end; ++u, ++k) {
+                        if (k & 1)
+                            l2_lookup_step<1, NB1, 1, ABS>(a, u, u_end, k, slab0, lane, full0 + 8, empty0 + 8, off1,
+                                                           wr, acc1, ok);
+                        else
+                            l2_lookup_step<1, NB1, 0, ABS>(a, u, u_end, k, slab0, lane, full0, empty0, off1, wr,
+                                                           acc1, ok);
+                    }
                 }
             }
-        }
+        };
+        if ((sbase & 0x00FFFFFFu) == kDynSmemBase)
+            lookups(std::true_type{});
+        else
+            lookups(std::false_type{});
 #pragma unroll
         for (int rs = 0; rs < kSlabsPerWarp; ++rs)
 #pragma unroll
