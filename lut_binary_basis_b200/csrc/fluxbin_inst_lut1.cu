@@ -13,10 +13,10 @@ template <int LW>
 KernelFn pick_l1(int nb0, int nb1) {
 #define FB_L1_NB1(NB0)                                         \
     switch (nb1) {                                             \
-        case 0: return &fluxbin_lut1_kernel<NB0, 0, LW>;      \
-        case 1: return &fluxbin_lut1_kernel<NB0, 1, LW>;      \
-        case 2: return &fluxbin_lut1_kernel<NB0, 2, LW>;      \
-        case 4: return &fluxbin_lut1_kernel<NB0, 4, LW>;      \
+        case 0: return &fluxbin_lut1_kernel<NB0, 0, LW, 2>;   \
+        case 1: return &fluxbin_lut1_kernel<NB0, 1, LW, 2>;   \
+        case 2: return &fluxbin_lut1_kernel<NB0, 2, LW, 2>;   \
+        case 4: return &fluxbin_lut1_kernel<NB0, 4, LW, 2>;   \
         default: return nullptr;                               \
     }
     switch (nb0) {

@@ -38,13 +38,13 @@
 
 namespace fluxbin {
 
-template <int LW>
+template <int LW, int SPW = kSlabsPerWarp>
 struct L1Geom {
     static constexpr int kLookupWarps = LW;
     static constexpr int kBuildWarps = LW / 4;
     static constexpr int kBuildThreads = kBuildWarps * kLanes;
     static constexpr int kThreads = (LW + kBuildWarps) * kLanes;
-    static constexpr int kSlabs = LW * kSlabsPerWarp;
+    static constexpr int kSlabs = LW * SPW;
     static constexpr int kRows = kSlabs * kLanes;
     static constexpr int kSlots = 256;                          // products per unit (32 tables x 8 bits)
     static constexpr int kSlotsPerThread = kSlots / kBuildThreads;
@@ -180,24 +180,28 @@ __device__ __forceinline__ void l1_lookup_unit(const uint4 (&w)[2], const Offset
 }
 
 // Lookup warps: one unit of branch BR in stage H (the k-th unit of the CTA).
-template <int BR, int NB, int H, bool ABS>
+// The packed words travel in a ring of D register sets per slab: a slab's
+// words for unit u + D are requested as soon as its unit-u lookups are done.
+template <int BR, int NB, int H, bool ABS, int SPW, int D>
 __device__ __forceinline__ void l1_lookup_step(const KernelArgs& a, int u, int u_end, int k, int slab0, int lane,
                                                uint32_t full_bar, uint32_t empty_bar, const Offsets<8>& off,
-                                               uint4 (&wr)[2][kSlabsPerWarp][2], float (&acc)[kSlabsPerWarp][NB],
-                                               bool& ok) {
+                                               uint4 (&wr)[D][SPW][2], float (&acc)[SPW][NB], bool& ok) {
+    constexpr int RS = D == 2 ? H : 0;
     if (ok) ok = l1_mbar_wait(full_bar, (uint32_t)((k >> 1) & 1));
 #pragma unroll
-    for (int rs = 0; rs < kSlabsPerWarp; ++rs) {
-        l1_lookup_unit<NB, H, ABS>(wr[H][rs], off, acc[rs]);
-        if (u + 2 < u_end) load_unit_slab<8, 1>(a, u + 2, slab0 + rs, lane, wr[H][rs]);
+    for (int rs = 0; rs < SPW; ++rs) {
+        l1_lookup_unit<NB, H, ABS>(wr[RS][rs], off, acc[rs]);
+        if (u + D < u_end) load_unit_slab<8, 1>(a, u + D, slab0 + rs, lane, wr[RS][rs]);
     }
     __syncwarp();
     if (lane == 0) l1_mbar_arrive(empty_bar);
 }
 
-template <int NB0, int NB1, int LW>
-__global__ void __launch_bounds__(L1Geom<LW>::kThreads, LW == 16 ? 1 : 2) fluxbin_lut1_kernel(const KernelArgs a) {
-    using G = L1Geom<LW>;
+template <int NB0, int NB1, int LW, int SPW>
+__global__ void __launch_bounds__(L1Geom<LW, SPW>::kThreads, LW == 16 ? 1 : 2)
+    fluxbin_lut1_kernel(const KernelArgs a) {
+    using G = L1Geom<LW, SPW>;
+    constexpr int D = SPW >= 4 ? 1 : 2;   // units of packed words held ahead per slab
     constexpr int NB1E = NB1 > 0 ? NB1 : 1;
     const int tid = threadIdx.x, warp = tid / kLanes, lane = tid % kLanes;
     const int ks = blockIdx.x % a.n_ks;
@@ -221,33 +225,54 @@ __global__ void __launch_bounds__(L1Geom<LW>::kThreads, LW == 16 ? 1 : 2) fluxbi
     __syncthreads();
 
     bool ok = true;
-    float tot[kSlabsPerWarp] = {0.f, 0.f};
-    const int slab0 = rg * G::kSlabs + warp * kSlabsPerWarp;
+    float tot[SPW];
+#pragma unroll
+    for (int rs = 0; rs < SPW; ++rs) tot[rs] = 0.f;
+    const int slab0 = rg * G::kSlabs + warp * SPW;
 
     if (warp < LW) {
         // ---------------- lookup warps ----------------
-        uint4 wr[2][kSlabsPerWarp][2];
-        __half sc0[kSlabsPerWarp][NB0], sc1[kSlabsPerWarp][NB1E];
+        uint4 wr[D][SPW][2];
+        __half sc0[SPW][NB0], sc1[SPW][NB1E];
         Offsets<8> off;
         off.template load<NB0, 0>(lane);
+        // Row scales of the lane's rows (kept as loaded, converted where
+        // applied): requested before the wait with D = 2, with the last unit
+        // otherwise (registers are tight with four slabs per warp).
+        auto fetch_scales = [&]() {
+#pragma unroll
+            for (int rs = 0; rs < SPW; ++rs) {
+                const int row = (slab0 + rs) * kLanes + lane;
+#pragma unroll
+                for (int q = 0; q < NB0; ++q) {
+                    const int kb = (q + lane / (32 / NB0)) % NB0;
+                    sc0[rs][q] = row < a.M ? a.br[0].r[(int64_t)kb * a.M + row] : __float2half(0.f);
+                }
+#pragma unroll
+                for (int q = 0; q < NB1E; ++q) {
+                    const int kb = (q + lane / (32 / NB1E)) % NB1E;
+                    sc1[rs][q] = (NB1 > 0 && row < a.M && a.br[1].units > 0) ? a.br[1].r[(int64_t)kb * a.M + row]
+                                                                            : __float2half(0.f);
+                }
+            }
+        };
         auto fetch = [&]() {
 #pragma unroll
-            for (int d = 0; d < 2; ++d)
+            for (int d = 0; d < D; ++d)
                 if (u_begin + d < u_end) {
 #pragma unroll
-                    for (int rs = 0; rs < kSlabsPerWarp; ++rs)
+                    for (int rs = 0; rs < SPW; ++rs)
                         load_unit_slab<8, 1>(a, u_begin + d, slab0 + rs, lane, wr[d][rs]);
                 }
-            fetch_row_scales<NB0>(a, a.br[0], slab0, lane, sc0);
-            if constexpr (NB1 > 0) fetch_row_scales<NB1>(a, a.br[1], slab0, lane, sc1);
+            if (D == 2 || u_end - u_begin <= 1) fetch_scales();
         };
         if (early) fetch();
         asm volatile("griddepcontrol.wait;" ::: "memory");
         if (!early) fetch();
 
-        float acc0[kSlabsPerWarp][NB0], acc1[kSlabsPerWarp][NB1E];
+        float acc0[SPW][NB0], acc1[SPW][NB1E];
 #pragma unroll
-        for (int rs = 0; rs < kSlabsPerWarp; ++rs) {
+        for (int rs = 0; rs < SPW; ++rs) {
 #pragma unroll
             for (int q = 0; q < NB0; ++q) acc0[rs][q] = 0.f;
 #pragma unroll
@@ -258,11 +283,13 @@ __global__ void __launch_bounds__(L1Geom<LW>::kThreads, LW == 16 ? 1 : 2) fluxbi
             if constexpr (ABS) off.set_rank_byte(sbase & 0xFF000000u);
             int k = 0;
             for (int u = u_begin; u < min(u_end, U0); ++u, ++k) {
+                if (D == 1 && u + 1 == u_end && u > u_begin) fetch_scales();
                 if (k & 1)
-                    l1_lookup_step<0, NB0, 1, ABS>(a, u, u_end, k, slab0, lane, full0 + 8, empty0 + 8, off, wr, acc0,
-                                                   ok);
+                    l1_lookup_step<0, NB0, 1, ABS, SPW, D>(a, u, u_end, k, slab0, lane, full0 + 8, empty0 + 8, off,
+                                                           wr, acc0, ok);
                 else
-                    l1_lookup_step<0, NB0, 0, ABS>(a, u, u_end, k, slab0, lane, full0, empty0, off, wr, acc0, ok);
+                    l1_lookup_step<0, NB0, 0, ABS, SPW, D>(a, u, u_end, k, slab0, lane, full0, empty0, off, wr, acc0,
+                                                           ok);
             }
             if constexpr (NB1 > 0) {
                 if (max(u_begin, U0) < u_end) {
@@ -270,12 +297,13 @@ __global__ void __launch_bounds__(L1Geom<LW>::kThreads, LW == 16 ? 1 : 2) fluxbi
                     off1.template load<NB1, 0>(lane);
                     if constexpr (ABS) off1.set_rank_byte(sbase & 0xFF000000u);
                     for (int u = max(u_begin, U0); u < u_end; ++u, ++k) {
+                        if (D == 1 && u + 1 == u_end && u > u_begin) fetch_scales();
                         if (k & 1)
-                            l1_lookup_step<1, NB1, 1, ABS>(a, u, u_end, k, slab0, lane, full0 + 8, empty0 + 8, off1,
-                                                           wr, acc1, ok);
+                            l1_lookup_step<1, NB1, 1, ABS, SPW, D>(a, u, u_end, k, slab0, lane, full0 + 8, empty0 + 8,
+                                                                   off1, wr, acc1, ok);
                         else
-                            l1_lookup_step<1, NB1, 0, ABS>(a, u, u_end, k, slab0, lane, full0, empty0, off1, wr,
-                                                           acc1, ok);
+                            l1_lookup_step<1, NB1, 0, ABS, SPW, D>(a, u, u_end, k, slab0, lane, full0, empty0, off1,
+                                                                   wr, acc1, ok);
                     }
                 }
             }
@@ -285,7 +313,7 @@ __global__ void __launch_bounds__(L1Geom<LW>::kThreads, LW == 16 ? 1 : 2) fluxbi
         else
             lookups(std::false_type{});
 #pragma unroll
-        for (int rs = 0; rs < kSlabsPerWarp; ++rs) {
+        for (int rs = 0; rs < SPW; ++rs) {
 #pragma unroll
             for (int q = 0; q < NB0; ++q) tot[rs] = fmaf(__half2float(sc0[rs][q]), acc0[rs][q], tot[rs]);
             if constexpr (NB1 > 0) {
@@ -370,14 +398,14 @@ __global__ void __launch_bounds__(L1Geom<LW>::kThreads, LW == 16 ? 1 : 2) fluxbi
     if (!ok) {
         atomicOr(a.err, 4u);
 #pragma unroll
-        for (int rs = 0; rs < kSlabsPerWarp; ++rs) tot[rs] = __int_as_float(0x7fc00000);
+        for (int rs = 0; rs < SPW; ++rs) tot[rs] = __int_as_float(0x7fc00000);
     }
     const bool lookup_warp = warp < LW;
     const int row0 = rg * G::kRows;
     if (a.n_ks == 1) {
         if (lookup_warp) {
 #pragma unroll
-            for (int rs = 0; rs < kSlabsPerWarp; ++rs) {
+            for (int rs = 0; rs < SPW; ++rs) {
                 const int i = (slab0 + rs) * kLanes + lane;
                 if (i < a.M) store_y(a, 0, i, tot[rs]);
             }
@@ -395,8 +423,8 @@ __global__ void __launch_bounds__(L1Geom<LW>::kThreads, LW == 16 ? 1 : 2) fluxbi
         const uint32_t red = sbase + G::kRedOff;
         if (lookup_warp) {
 #pragma unroll
-            for (int rs = 0; rs < kSlabsPerWarp; ++rs) {
-                const int lr = (warp * kSlabsPerWarp + rs) * kLanes + lane;
+            for (int rs = 0; rs < SPW; ++rs) {
+                const int lr = (warp * SPW + rs) * kLanes + lane;
                 const int owner = lr / chunk, j = lr % chunk;
                 st_dsmem_f32(red + (uint32_t)(rank * chunk + j) * 4u, (uint32_t)owner, tot[rs]);
             }
@@ -418,7 +446,7 @@ __global__ void __launch_bounds__(L1Geom<LW>::kThreads, LW == 16 ? 1 : 2) fluxbi
     // the row group to arrive finishes the sum, writes y and re-zeroes it.
     if (lookup_warp) {
 #pragma unroll
-        for (int rs = 0; rs < kSlabsPerWarp; ++rs) {
+        for (int rs = 0; rs < SPW; ++rs) {
             const int i = (slab0 + rs) * kLanes + lane;
             if (i < a.M) red_add_f32(a.ws_acc + i, tot[rs]);
         }
