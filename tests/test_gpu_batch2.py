@@ -94,3 +94,34 @@ def test_pair_tables_error_is_table_rounding_sized():
         e_gpu = np.linalg.norm(got[b] - exact[b])
         e_q = np.linalg.norm(q16[b] - exact[b])
         assert e_gpu <= 4 * e_q + 1e-6 * np.linalg.norm(exact[b])
+
+
+@pytest.mark.parametrize("M,N,n_sal,B", [(16400, 9000, 8300, 1), (3000, 5000, 2600, 4), (2000, 3000, 1200, 7)],
+                         ids=["batch1_large", "pairs_b4", "pairs_b7"])
+def test_lut_gemv_gathered_branch_on_new_kernels(M, N, n_sal, B):
+    """fluxbin_lut_gemv on a gathered column set (the salient branch alone,
+    Virtual Columnar Mapping) through the warp-specialised batch-1 kernel
+    (M * ncols >= 2^27) and the batch-pair kernel, with an out-of-range
+    column index contributing nothing."""
+    import dataclasses
+    sp = spec(M, N, 1, 2, n_sal, 8)
+    layer = synth.make_layer(sp, [640, M, B])
+    x = synth.make_x(sp, B, [641, M, B])
+    words, swords = fluxbin.fluxbin_pack(fluxbin.LayerDesc.of(sp), layer.signs, layer.sal_signs, layer.sal_idx)
+    sw = torch.from_numpy(swords.view(np.int32)).cuda()
+    rs, cs = torch.from_numpy(layer.rs).cuda(), torch.from_numpy(layer.cs).cuda()
+    xd = torch.from_numpy(x).cuda()
+    ws = fluxbin.new_workspace(M, B)
+    only_sal = dataclasses.replace(layer, c=np.zeros_like(layer.c))
+    for bad in (False, True):
+        idx = layer.sal_idx.copy()
+        cs_ref = layer.cs.copy()
+        if bad:
+            idx[7] = N + 3
+            cs_ref[:, 7] = 0
+        y = torch.full((B, M), float("nan"), dtype=torch.float32, device="cuda")
+        fluxbin.fluxbin_lut_gemv(M, N, n_sal, 2, 8, 0, sw, rs, cs, torch.from_numpy(idx).cuda(), xd, B, y,
+                                 fluxbin.FLAG_Y_FP32, ws)
+        torch.cuda.synchronize()
+        ref = oracle.linear(dataclasses.replace(only_sal, cs=cs_ref), x)
+        assert_close(y.cpu().numpy().astype(np.float64), ref, only_sal, x)

@@ -81,3 +81,29 @@ def test_static_scratch_rejects_layers_beyond_its_size():
     st = L.fluxbin_linear_static_scratch(ctypes.byref(desc), 0x1000, 0x2000, 0x3000, 0, 0, 0, 0, 0x4000, 16, 0x5000,
                                          fluxbin.FLAG_Y_FP32, None)
     assert st == -8
+
+
+@pytest.mark.parametrize("sp,B", [
+    (LayerSpec("large_b1", 16400, 8192, 2, 2, 246, 8), 1),   # warp-specialised batch-1 kernel
+    (LayerSpec("pairs", 5000, 4096, 2, 1, 205, 8), 6),       # batch pairs on fp16-pair tables
+])
+def test_static_scratch_on_the_new_kernels(sp, B):
+    """The static scratch behind the batch-1 and batch-pair kernels, whose
+    plans split one CTA per SM through the scratch: two calls in a row, each
+    checked against the oracle."""
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    torch.cuda.set_device(0)
+    layer = synth.make_layer(sp, [125, sp.M, B])
+    x = synth.make_x(sp, B, [126, sp.M, B])
+    d = fluxbin.DeviceLayer.from_host(layer)
+    xd = torch.from_numpy(x).cuda()
+    exact = oracle.linear(layer, x)
+    for call in range(2):
+        y = torch.full((B, sp.M), float("nan"), dtype=torch.float32, device="cuda")
+        fluxbin.fluxbin_linear_static_scratch(d.desc, d.words, d.r, d.c, d.swords, d.rs, d.cs, d.idx, xd, B, y,
+                                              fluxbin.FLAG_Y_FP32)
+        torch.cuda.synchronize()
+        got = y.cpu().numpy().astype(np.float64)
+        assert np.all(np.isfinite(got)), f"call {call}"
+        close(got, exact, layer, x)
