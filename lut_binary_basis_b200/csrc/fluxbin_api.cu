@@ -199,49 +199,46 @@ struct Plan {
     bool cluster = false;
 };
 
-// Row groups of 512 rows times batch chunks fix the number of CTA groups; the
-// units are split over up to 16 CTAs per group forming a cluster whose
-// partials are reduced in DSMEM, choosing the widest split for which every
-// cluster is resident at once, up to one CTA per CTA slot of the GPU (two per
-// SM: one CTA's table build then overlaps the other's lookups).  When that
-// leaves most SMs idle (few rows, long rows) the units are split as widely
-// as the SMs allow and reduced through the workspace.
+// Row groups (of the CTA's rows) times batch chunks fix the number of CTA
+// groups; the units of a group are split over several CTAs, either a cluster
+// whose partials are reduced in DSMEM (the widest split for which every
+// cluster is resident at once, up to one CTA per CTA slot of the GPU) or, with
+// a workspace from the caller, a split reduced through the workspace.
+//
+// The workspace split is as wide as one CTA per slot allows, then narrowed to
+// as few CTAs as give the same units per CTA; it is taken unless a resident
+// cluster split leaves each CTA as few units.  A call's time is set by its
+// slowest CTA, i.e. by the units per CTA and by how many CTAs share an SM:
+// clusters must sit inside one GPU processing cluster, which caps their width
+// and places them unevenly.  Measured on B200 at batch 1 (graph of calls):
+// 4096x4096 5.37 -> 4.01 us (one cluster of 16 per row group against 17 CTAs
+// through the workspace), 4096x4096 at 2.75 bits with block-wise scales 7.75
+// -> 5.35 us, 4096x11008 at 2.75 bits 11.81 -> 9.89 us, 8192x28672 at mu = 4
+// 55.8 -> 41.7 us; 4096x4096 at batch 2 6.52 -> 5.45 us.
 Plan make_plan(KernelFn fn, int dev, const CtaShape& cs, int64_t Ms, int64_t U, int n_bc, const DeviceInfo& di,
                const FuncInfo& fi, bool have_ws, bool fill_gpu = false) {
     Plan p;
     p.n_rg = (int)((Ms + cs.slabs - 1) / cs.slabs);
     const int64_t groups = (int64_t)p.n_rg * n_bc;
     const int64_t slots = (int64_t)di.sm_count * fi.blocks_per_sm;
+    const size_t smem = cs.smem;
+    const int64_t ks_cap = std::min<int64_t>(U, slots / groups);
+    const int64_t units_wide = ks_cap >= 1 ? (U + ks_cap - 1) / ks_cap : U;
+    const int64_t ks_wide = (U + units_wide - 1) / units_wide;
+    const bool wide_ok = have_ws && ks_wide >= 2;
+
     int64_t want = slots / groups;
     if (want > U) want = U;
     if (want > kMaxCluster) want = kMaxCluster;
-    const size_t smem = cs.smem;
-    // Long rows on few row groups: a split wider than a cluster, reduced
-    // through the workspace, shortens each CTA's chain of units by more than
-    // the workspace reduction costs once a cluster would leave every CTA at
-    // least two more units (B200, batch 1: 4096x11008 8.5 us with a 30-way
-    // workspace split against 10.6 us with 16-CTA clusters; 4096x4096 and
-    // 11008x4096, where clusters leave 2-3 units per CTA, are faster with
-    // clusters).  Up to 85% of the slots (the rest stays free for the next
-    // call's early CTAs), then as few CTAs as give the same units per CTA.
-    // Only with a workspace from the caller.
-    const int64_t ks_cap = std::min<int64_t>(U, (slots * 17) / (20 * groups));
-    const int64_t units_wide = ks_cap >= 1 ? (U + ks_cap - 1) / ks_cap : U;
-    const int64_t ks_wide = (U + units_wide - 1) / units_wide;
-    if (have_ws && want >= 1 && ks_wide > kMaxCluster && (U + want - 1) / want >= units_wide + 2) {
-        p.n_ks = (int)ks_wide;
-        p.cluster = false;
-        return p;
-    }
     for (int64_t ks = want; ks >= 2; --ks) {
         if (have_ws && groups * ks * 2 < di.sm_count) break;  // too few CTAs: use the workspace instead
         if (max_active_clusters(fn, dev, (int)ks, smem, cs.threads) >= groups) {
+            if (wide_ok && units_wide < (U + ks - 1) / ks) break;  // the workspace split is shorter
             p.n_ks = (int)ks;
             p.cluster = true;
             // One CTA per SM: a cluster size that fits fewer CTAs than the
-            // GPU has slots (clusters must sit inside one GPU processing
-            // cluster) leaves SMs idle; split one CTA per slot through the
-            // workspace instead when that fills at least an eighth more.
+            // GPU has slots leaves SMs idle; split one CTA per slot through
+            // the workspace instead when that fills at least an eighth more.
             const int64_t ks_ws = std::min<int64_t>(U, slots / groups);
             if (fill_gpu && have_ws && ks_ws * 8 >= ks * 9) {
                 p.n_ks = (int)ks_ws;
@@ -249,6 +246,11 @@ Plan make_plan(KernelFn fn, int dev, const CtaShape& cs, int64_t Ms, int64_t U, 
             }
             return p;
         }
+    }
+    if (wide_ok) {
+        p.n_ks = (int)ks_wide;
+        p.cluster = false;
+        return p;
     }
     if (groups * 2 >= di.sm_count || U <= 1 || !have_ws) {
         p.n_ks = 1;  // enough row groups (or no workspace): no split at all

@@ -868,21 +868,34 @@ __global__ void __launch_bounds__(kThreads, MB) fluxbin_lut_kernel(const KernelA
         for (int b = 0; b < BT; ++b)
             if (b0 + b < a.B) red_add_f32(a.ws_acc + (int64_t)(b0 + b) * a.Mp + i, tot[rs][b]);
     }
-    __threadfence();
     __syncthreads();
     __shared__ unsigned int s_last;
     unsigned int* cnt = a.ws_cnt + (rg * a.n_bc + bc);
-    if (tid == 0) s_last = (atomicAdd(cnt, 1u) == (unsigned)(a.n_ks - 1)) ? 1u : 0u;
+    if (tid == 0) {
+        __threadfence();   // cumulative: orders the CTA's adds (barrier above) before the count
+        s_last = (atomicAdd(cnt, 1u) == (unsigned)(a.n_ks - 1)) ? 1u : 0u;
+        __threadfence();
+    }
     __syncthreads();
     if (!s_last) return;
-    __threadfence();
-    for (int e = tid; e < kRowsPerCta * BT; e += kThreads) {
-        const int b = e / kRowsPerCta, i = row0 + e % kRowsPerCta;
-        if (i >= a.M || b0 + b >= a.B) continue;
-        float* p = a.ws_acc + (int64_t)(b0 + b) * a.Mp + i;
-        const float val = __ldcg(p);
-        __stcg(p, 0.f);
-        store_y(a, b0 + b, i, val);
+    // each lane finishes its own rows, all loads before the first store
+    float val[kSlabsPerWarp][BT];
+#pragma unroll
+    for (int rs = 0; rs < kSlabsPerWarp; ++rs) {
+        const int i = (slab0 + rs) * kLanes + lane;
+#pragma unroll
+        for (int b = 0; b < BT; ++b)
+            val[rs][b] = (i < a.M && b0 + b < a.B) ? __ldcg(a.ws_acc + (int64_t)(b0 + b) * a.Mp + i) : 0.f;
+    }
+#pragma unroll
+    for (int rs = 0; rs < kSlabsPerWarp; ++rs) {
+        const int i = (slab0 + rs) * kLanes + lane;
+#pragma unroll
+        for (int b = 0; b < BT; ++b)
+            if (i < a.M && b0 + b < a.B) {
+                __stcg(a.ws_acc + (int64_t)(b0 + b) * a.Mp + i, 0.f);
+                store_y(a, b0 + b, i, val[rs][b]);
+            }
     }
     if (tid == 0) *cnt = 0u;
 }

@@ -444,6 +444,9 @@ __global__ void __launch_bounds__(L1Geom<LW, SPW>::kThreads, LW == 16 ? 1 : 2)
     }
     // Split-K through the workspace: add this CTA's partials; the last CTA of
     // the row group to arrive finishes the sum, writes y and re-zeroes it.
+    // The CTA barrier orders every thread's adds before thread 0's fence and
+    // counter increment (the fence is cumulative), so one fence per CTA
+    // publishes them.
     if (lookup_warp) {
 #pragma unroll
         for (int rs = 0; rs < SPW; ++rs) {
@@ -451,21 +454,33 @@ __global__ void __launch_bounds__(L1Geom<LW, SPW>::kThreads, LW == 16 ? 1 : 2)
             if (i < a.M) red_add_f32(a.ws_acc + i, tot[rs]);
         }
     }
-    __threadfence();
     __syncthreads();
     unsigned int* cnt = a.ws_cnt + rg;
     uint32_t& s_last = smem_at<uint32_t>(G::kBarOff + 32);
-    if (tid == 0) s_last = (atomicAdd(cnt, 1u) == (unsigned)(a.n_ks - 1)) ? 1u : 0u;
+    if (tid == 0) {
+        __threadfence();
+        s_last = (atomicAdd(cnt, 1u) == (unsigned)(a.n_ks - 1)) ? 1u : 0u;
+        __threadfence();
+    }
     __syncthreads();
     if (!s_last) return;
-    __threadfence();
-    for (int e = tid; e < G::kRows; e += G::kThreads) {
-        const int i = row0 + e;
-        if (i >= a.M) continue;
-        float* p = a.ws_acc + i;
-        const float val = __ldcg(p);
-        __stcg(p, 0.f);
-        store_y(a, 0, i, val);
+    // Each lookup lane finishes its own rows: every load is issued before the
+    // first store, so the sums take one round trip.
+    if (lookup_warp) {
+        float val[SPW];
+#pragma unroll
+        for (int rs = 0; rs < SPW; ++rs) {
+            const int i = (slab0 + rs) * kLanes + lane;
+            val[rs] = i < a.M ? __ldcg(a.ws_acc + i) : 0.f;
+        }
+#pragma unroll
+        for (int rs = 0; rs < SPW; ++rs) {
+            const int i = (slab0 + rs) * kLanes + lane;
+            if (i < a.M) {
+                __stcg(a.ws_acc + i, 0.f);
+                store_y(a, 0, i, val[rs]);
+            }
+        }
     }
     if (tid == 0) *cnt = 0u;
 }

@@ -291,21 +291,30 @@ __global__ void __launch_bounds__(L1hGeom<LW, SPW>::kThreads, 1)
         const int row = (slab0 + rs) * kLanes + lane;
         if (row < a.M) red_add_f32(a.ws_acc + row, tot[rs]);
     }
-    __threadfence();
     __syncthreads();
     unsigned int* cnt = a.ws_cnt + rg;
     uint32_t& s_last = smem_at<uint32_t>(G::kBarOff + 32);
-    if (tid == 0) s_last = (atomicAdd(cnt, 1u) == (unsigned)(a.n_ks - 1)) ? 1u : 0u;
+    if (tid == 0) {
+        __threadfence();   // cumulative: orders the CTA's adds (barrier above) before the count
+        s_last = (atomicAdd(cnt, 1u) == (unsigned)(a.n_ks - 1)) ? 1u : 0u;
+        __threadfence();
+    }
     __syncthreads();
     if (!s_last) return;
-    __threadfence();
-    for (int e = tid; e < G::kRows; e += G::kThreads) {
-        const int i = row0 + e;
-        if (i >= a.M) continue;
-        float* p = a.ws_acc + i;
-        const float val = __ldcg(p);
-        __stcg(p, 0.f);
-        store_y(a, 0, i, val);
+    // each lane finishes its own rows, all loads before the first store
+    float val[SPW];
+#pragma unroll
+    for (int rs = 0; rs < SPW; ++rs) {
+        const int row = (slab0 + rs) * kLanes + lane;
+        val[rs] = row < a.M ? __ldcg(a.ws_acc + row) : 0.f;
+    }
+#pragma unroll
+    for (int rs = 0; rs < SPW; ++rs) {
+        const int row = (slab0 + rs) * kLanes + lane;
+        if (row < a.M) {
+            __stcg(a.ws_acc + row, 0.f);
+            store_y(a, 0, row, val[rs]);
+        }
     }
     if (tid == 0) *cnt = 0u;
 }

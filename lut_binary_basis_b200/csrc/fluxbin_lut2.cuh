@@ -416,21 +416,36 @@ __global__ void __launch_bounds__(L2Geom<LW>::kThreads, 1) fluxbin_lut2_kernel(c
                 if (i < a.M && b0 + r < a.B) red_add_f32(a.ws_acc + (int64_t)(b0 + r) * a.Mp + i, tot[rs][r]);
         }
     }
-    __threadfence();
     __syncthreads();
     unsigned int* cnt = a.ws_cnt + (rg * a.n_bc + bp);
     uint32_t& s_last = smem_at<uint32_t>(G::kBarOff + 32);
-    if (tid == 0) s_last = (atomicAdd(cnt, 1u) == (unsigned)(a.n_ks - 1)) ? 1u : 0u;
+    if (tid == 0) {
+        __threadfence();   // cumulative: orders the CTA's adds (barrier above) before the count
+        s_last = (atomicAdd(cnt, 1u) == (unsigned)(a.n_ks - 1)) ? 1u : 0u;
+        __threadfence();
+    }
     __syncthreads();
     if (!s_last) return;
-    __threadfence();
-    for (int e = tid; e < 2 * G::kRows; e += G::kThreads) {
-        const int r = e / G::kRows, i = row0 + e % G::kRows;
-        if (i >= a.M || b0 + r >= a.B) continue;
-        float* p = a.ws_acc + (int64_t)(b0 + r) * a.Mp + i;
-        const float val = __ldcg(p);
-        __stcg(p, 0.f);
-        store_y(a, b0 + r, i, val);
+    // each lookup lane finishes its own rows, all loads before the first store
+    if (lookup_warp) {
+        float val[kSlabsPerWarp][2];
+#pragma unroll
+        for (int rs = 0; rs < kSlabsPerWarp; ++rs) {
+            const int i = (slab0 + rs) * kLanes + lane;
+#pragma unroll
+            for (int r = 0; r < 2; ++r)
+                val[rs][r] = (i < a.M && b0 + r < a.B) ? __ldcg(a.ws_acc + (int64_t)(b0 + r) * a.Mp + i) : 0.f;
+        }
+#pragma unroll
+        for (int rs = 0; rs < kSlabsPerWarp; ++rs) {
+            const int i = (slab0 + rs) * kLanes + lane;
+#pragma unroll
+            for (int r = 0; r < 2; ++r)
+                if (i < a.M && b0 + r < a.B) {
+                    __stcg(a.ws_acc + (int64_t)(b0 + r) * a.Mp + i, 0.f);
+                    store_y(a, b0 + r, i, val[rs][r]);
+                }
+        }
     }
     if (tid == 0) *cnt = 0u;
 }
