@@ -697,11 +697,13 @@ int run(int32_t M, int32_t N, int mu, const BranchIn& g, const BranchIn* s, cons
     // batch 1, mu = 8, per-row scales: the table precompute as its own kernel
     // when asked for (and the workspace has room for the tables); otherwise,
     // for large layers, the warp-specialised kernel (B200, batch 1:
-    // 28672x8192 25.3 -> 22.0 us, 8192x28672 29.1 -> 21.2 us; 11008x4096
-    // 8.0 -> 8.6 us and 4096x4096 5.4 -> 6.0 us, which stay on the kernel
-    // below).  With the precompute as its own kernel the same layers measured
-    // 25.2 and 31.3 us: the lookups alone took longer than the warp-specialised
-    // kernel with its in-CTA build, and the precompute ran before them.
+    // 28672x8192 25.3 -> 22.0 us, 8192x28672 29.1 -> 21.2 us).  From 2^25
+    // weights with a workspace (11008x4096 and 4096x11008 7.0 -> 6.7 us with
+    // the workspace split of both kernels), from 2^27 without; 4096x4096
+    // stays on the kernel below (4.0 against 4.2 us).  With the precompute as
+    // its own kernel the large layers measured 25.2 and 31.3 us: the lookups
+    // alone took longer than the warp-specialised kernel with its in-CTA
+    // build, and the precompute ran before them.
     if (B == 1 && mu == 8 && g.rgroup == 0 && (!nb1 || s->rgroup == 0)) {
         const int64_t U = branch_units(g.ncols, g.nb, mu) + (nb1 ? branch_units(s->ncols, nb1, mu) : 0);
         if (flags & kFlagSeparateTables) {
@@ -709,7 +711,8 @@ int run(int32_t M, int32_t N, int mu, const BranchIn& g, const BranchIn* s, cons
             if (!aligned(ws, 16)) return FLUXBIN_ERR_MISALIGNED;
             return run_lut1h(M, N, g, s, nb1, d_x, d_y, flags & ~kFlagSeparateTables, ws, stream, uses_ws);
         }
-        if ((int64_t)M * N >= ((int64_t)1 << 27))
+        const bool ws_ok = ws && ws_bytes >= workspace_bytes_for(M, 1) && aligned(ws, 16);
+        if ((int64_t)M * N >= ((int64_t)1 << (ws_ok ? 25 : 27)))
             return run_lut1(M, N, g, s, nb1, d_x, d_y, flags, ws, ws_bytes, stream, uses_ws);
     } else if (flags & kFlagSeparateTables) {
         return FLUXBIN_ERR_UNSUPPORTED;

@@ -1,14 +1,15 @@
 """GPU parity of the batch-1, mu = 8 kernels against the fp64 oracle.
 
-Large layers (M * N >= 2^27) at batch 1 run the warp-specialised kernel
-(builder warps fill a two-stage table ring, lookup warps consume it through
-mbarriers); FLUXBIN_FLAG_SEPARATE_TABLES runs the table precompute as a kernel
-of its own followed by the lookup-only kernel fed by bulk copies.  Both are
-compared with the oracle on every output row, with and without a caller
-workspace (the plans differ: clusters or a split through the workspace), on
-ragged shapes and every base count the kernels are built for.  Same
-tolerance as the other parity tests; exact-arithmetic layers must match bit
-for bit.
+Large layers at batch 1 (M * N >= 2^27, or >= 2^25 with a workspace) run the
+warp-specialised kernel (builder warps fill a two-stage table ring, lookup
+warps consume it through mbarriers); FLUXBIN_FLAG_SEPARATE_TABLES runs the
+table precompute as a kernel of its own followed by the lookup-only kernel
+fed by bulk copies.  Both are compared with the oracle on every output row,
+with and without a caller workspace (the plans differ: clusters or a split
+through the workspace; mid-sized layers without one stay on the original
+kernel), on ragged shapes and every base count the kernels are built for.
+Same tolerance as the other parity tests; exact-arithmetic layers must match
+bit for bit.
 """
 import numpy as np
 import pytest
@@ -55,6 +56,24 @@ LARGE = [
 @pytest.mark.parametrize("sp", LARGE, ids=lambda s: f"{s.M}x{s.N}_kb{s.Kb}_ks{s.Ks}")
 def test_large_layers_every_row(sp):
     assert sp.M * sp.N >= 1 << 27
+    _every_row(sp)
+
+
+MID = [
+    spec(11008, 4096, 2, 1, 205, 8),      # the 7B MLP shapes
+    spec(4096, 11008, 2, 1, 550, 8),
+    spec(6001, 5900, 1, 2, 300, 8),       # ragged rows and columns
+    spec(8192, 4097, 4, 0, 0, 8),
+]
+
+
+@pytest.mark.parametrize("sp", MID, ids=lambda s: f"{s.M}x{s.N}_kb{s.Kb}_ks{s.Ks}")
+def test_mid_layers_every_row(sp):
+    assert (1 << 25) <= sp.M * sp.N < (1 << 27)
+    _every_row(sp)
+
+
+def _every_row(sp):
     layer = synth.make_layer(sp, [500, sp.M, sp.N])
     x = synth.make_x(sp, 1, [501, sp.M])
     ref = oracle.linear(layer, x)
