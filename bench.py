@@ -18,8 +18,11 @@ are independent replicas (weak scaling).
 The same JSON line carries, under "configs", every other configuration
 timed the same way (the 4096 x 4096 projection; the 7B MLP shapes at batch
 1, 2, 4, 8; the 70B MLP shapes at mu = 8 and 4, batch 1 and 16), each with
-its graph-pipelined and serialised time per call, and under "stack" the
-32-layer 2.75-bit LLaMA-2-7B-shaped stack of linears under one CUDA graph.
+its graph-pipelined and serialised time per call, under "stack" the
+32-layer 2.75-bit LLaMA-2-7B-shaped stack of linears under one CUDA graph,
+and under "precompute_fusion" the batch-1 layer with its table precompute
+fused into the preceding RMS normalisation against the precompute as its
+own kernel and against the default path.
 
 --impl reference times the fp64 CPU oracle (all host cores) on the bounded
 sample of the headline layer that the cpu_baseline leg uses, in the same
@@ -433,6 +436,52 @@ def run_configs(device, l2, skip=None):
     return out
 
 
+def precompute_fusion_entry(spec, layer, device, wid, steps=50):
+    """Batch 1: the layer with its table precompute fused into the preceding
+    RMS normalisation (fluxbin_linear_rmsnorm, reading the un-normalised row),
+    against the precompute as its own kernel on an already normalised row
+    (FLUXBIN_FLAG_SEPARATE_TABLES) and against the library's default path;
+    µs per call in a CUDA graph of R dependent calls over R copies (L2-cold
+    like the other entries)."""
+    import numpy as np
+    import torch
+    from lut_binary_basis_b200 import fluxbin
+    copies, xs, ys, R = build_pool(layer, spec, 1, device, L2_BYTES, wid)
+    ws = copies[0].workspace(1)
+    gamma = torch.from_numpy(np.random.default_rng([wid, 77]).uniform(0.5, 1.5, spec.N).astype(np.float16)).to(device)
+    stream = torch.cuda.Stream(device)
+    ew = fluxbin.FLAG_EARLY_WEIGHTS
+    calls = {
+        "fused_rmsnorm_us": lambda i: copies[i].linear_rmsnorm(xs[i][0], gamma, 1e-5, ys[i], ew, ws, None, stream),
+        "separate_tables_us": lambda i: copies[i].linear(xs[i], ys[i], ew | fluxbin.FLAG_SEPARATE_TABLES, ws, stream),
+        "default_path_us": lambda i: copies[i].linear(xs[i], ys[i], ew, ws, stream),
+    }
+    out = {"layer": spec.name, "B": 1, "copies": R}
+    for name, fn in calls.items():
+        with torch.cuda.stream(stream):
+            for i in range(R):
+                fn(i)
+        stream.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for i in range(R):
+                fn(i)
+        out[name] = time_graph(g, stream, steps) / R * 1e6
+        del g
+    del copies, xs, ys
+    torch.cuda.empty_cache()
+    return out
+
+
+def run_precompute_fusion(device):
+    from lut_binary_basis_b200 import synth
+    out = {}
+    for wid, sp in ((HEADLINE_WID, headline_spec()), (1, synth.layer_7b_proj())):
+        layer = synth.make_layer(sp, synth.layer_key(wid, 0, 0))
+        out[sp.name] = precompute_fusion_entry(sp, layer, device, wid)
+    return out
+
+
 HEADLINE_WID = 3
 
 
@@ -571,6 +620,7 @@ def run_ours(args, rank, local_rank, world):
         if not args.headline_only:
             configs = run_configs(device, l2, skip={headline_name: headline_entry})
         stack = None if (args.headline_only or args.no_stack) else run_stack(args, device, summary=True)
+        fusion = None if args.headline_only else run_precompute_fusion(device)
         result = {
             "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": max_secs / args.steps * 1e3, "higher_is_better": True,
@@ -592,6 +642,7 @@ def run_ours(args, rank, local_rank, world):
             "clocks": clocks,
             "configs": configs,
             "stack": stack,
+            "precompute_fusion": fusion,
         }
         if cub and cub.get("us_per_call"):
             cub["lut_speedup_vs_dense"] = cub["us_per_call"] / us_per_call

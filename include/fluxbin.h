@@ -302,6 +302,41 @@ int fluxbin_linear(const fluxbin_layer_desc* desc,
                    void* stream);
 
 /*
+ * The layer with the table precompute fused into the element-wise operator
+ * that precedes it (LUT Tensor Core notes, Section 3.1.1: the precompute as
+ * an operator of its own, fused with the preceding element-wise operator).
+ * The operator is taken to be the RMS normalisation of a LLaMA-style block:
+ *   x = h (.) gamma / sqrt(mean_n(h[n]^2) + eps)
+ *   y (+)= W x
+ * for one activation row (batch 1).  The precompute kernel reads h, forms x
+ * in fp32 and builds every unit's tables from it (x is never rounded on the
+ * way to the tables); the lookup kernel of FLUXBIN_FLAG_SEPARATE_TABLES then
+ * runs on those tables.
+ *   d_h       fp16 [N], the un-normalised activation
+ *   d_gamma   fp16 [N], the normalisation weight
+ *   eps       >= 0, finite
+ *   d_x_out   fp16 [N] or NULL: if given, receives x rounded to fp16 (round to
+ *             nearest even), e.g. for the other layers that read the same x;
+ *             must not overlap d_h
+ *   flags     FLUXBIN_FLAG_ACCUMULATE, FLUXBIN_FLAG_Y_FP32,
+ *             FLUXBIN_FLAG_EARLY_WEIGHTS only
+ *   d_workspace, workspace_bytes   at least fluxbin_layer_workspace_bytes(desc, 1)
+ *             (the split-K scratch plus the table buffer), 16-byte aligned
+ * Other arguments as for fluxbin_linear.  Layers: mu = 8 with per-row scales
+ * in both branches (else UNSUPPORTED).  M == 0 returns FLUXBIN_OK without
+ * launching (x_out is then not written); N == 0 with M > 0 is BAD_SHAPE.
+ * Graph-capturable like fluxbin_linear.
+ * Errors: INVALID_ARG, BAD_SHAPE, MISALIGNED, UNSUPPORTED, WORKSPACE, CUDA.
+ */
+int fluxbin_linear_rmsnorm(const fluxbin_layer_desc* desc,
+                           const uint32_t* d_words, const uint16_t* d_r, const uint16_t* d_c,
+                           const uint32_t* d_swords, const uint16_t* d_rs, const uint16_t* d_cs,
+                           const int32_t* d_idx, const uint16_t* d_h, const uint16_t* d_gamma,
+                           float eps, uint16_t* d_x_out,
+                           void* d_y, uint32_t flags, void* d_workspace, size_t workspace_bytes,
+                           void* stream);
+
+/*
  * fluxbin_linear for callers that cannot allocate device memory.  (An
  * addition of this library; the FluxBin pages have no counterpart.)
  *

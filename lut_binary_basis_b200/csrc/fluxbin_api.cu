@@ -29,9 +29,9 @@ KernelFn select_kernel_lut2(int nb0, int nb1);
 int lut2_threads();
 int lut2_smem_bytes();
 int lut2_slabs();
-using TabKernelFn = void (*)(KernelArgs, float*);
+using TabKernelFn = void (*)(KernelArgs, float*, NormArgs);
 using HKernelFn = void (*)(KernelArgs, const float*);
-TabKernelFn select_tables_kernel(int nb0, int nb1);
+TabKernelFn select_tables_kernel(int nb0, int nb1, bool norm);
 HKernelFn select_kernel_lut1h(int spw, int nb0, int nb1);
 int lut1h_threads(int spw);
 int lut1h_smem_bytes(int spw);
@@ -566,7 +566,7 @@ int run_lut2(int32_t M, int32_t N, const BranchIn& g, const BranchIn* s, int nb1
 // then the lookups on the precomputed tables (fluxbin_lut1h.cuh).  2048 rows
 // per CTA when that plan keeps most SMs busy, else 1024.
 int run_lut1h(int32_t M, int32_t N, const BranchIn& g, const BranchIn* s, int nb1, const uint16_t* d_x, void* d_y,
-              uint32_t flags, void* ws, void* stream, int* uses_ws) {
+              uint32_t flags, void* ws, void* stream, int* uses_ws, const NormArgs* norm = nullptr) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return FLUXBIN_ERR_CUDA;
     KernelArgs a = {};
@@ -576,7 +576,7 @@ int run_lut1h(int32_t M, int32_t N, const BranchIn& g, const BranchIn* s, int nb
     DeviceInfo di;
     unsigned int* err = nullptr;
     HKernelFn fn = nullptr;
-    TabKernelFn tfn = select_tables_kernel(g.nb, nb1);
+    TabKernelFn tfn = select_tables_kernel(g.nb, nb1, norm != nullptr);
     Plan plan;
     int spw = 4;
     {
@@ -637,7 +637,7 @@ int run_lut1h(int32_t M, int32_t N, const BranchIn& g, const BranchIn* s, int nb
     tc.stream = static_cast<cudaStream_t>(stream);
     tc.attrs = attr;
     tc.numAttrs = 1;
-    cudaError_t le = cudaLaunchKernelEx(&tc, tfn, a, tables);
+    cudaError_t le = cudaLaunchKernelEx(&tc, tfn, a, tables, norm ? *norm : NormArgs{nullptr, 0.f, nullptr});
     if (le != cudaSuccess) return cuda_fail(le);
 
     cudaLaunchConfig_t cfg = {};
@@ -899,6 +899,49 @@ int fluxbin_linear(const fluxbin_layer_desc* desc, const uint32_t* d_words, cons
                    void* d_workspace, size_t workspace_bytes, void* stream) {
     return linear_impl(desc, d_words, d_r, d_c, d_swords, d_rs, d_cs, d_idx, d_x, B, d_y, flags, d_workspace,
                        workspace_bytes, stream, nullptr);
+}
+
+int fluxbin_linear_rmsnorm(const fluxbin_layer_desc* desc, const uint32_t* d_words, const uint16_t* d_r,
+                           const uint16_t* d_c, const uint32_t* d_swords, const uint16_t* d_rs, const uint16_t* d_cs,
+                           const int32_t* d_idx, const uint16_t* d_h, const uint16_t* d_gamma, float eps,
+                           uint16_t* d_x_out, void* d_y, uint32_t flags, void* d_workspace, size_t workspace_bytes,
+                           void* stream) {
+    const int st = validate_desc(desc);
+    if (st != FLUXBIN_OK) return st;
+    const fluxbin_layer_desc& d = *desc;
+    if (flags & ~(kFlagAccumulate | kFlagYFp32 | kFlagEarlyWeights)) return FLUXBIN_ERR_INVALID_ARG;
+    if (!(eps >= 0.f) || eps > 3.0e38f) return FLUXBIN_ERR_INVALID_ARG;   // negative, NaN or infinite
+    if (d.M == 0) return FLUXBIN_OK;
+    if (d.N == 0) return FLUXBIN_ERR_BAD_SHAPE;   // no mean of h^2 to take
+    if (!hoistable(d, 1)) return FLUXBIN_ERR_UNSUPPORTED;
+    if (!d_h || !d_gamma || !d_y) return FLUXBIN_ERR_INVALID_ARG;
+    if (has_salient(d) && !d_idx) return FLUXBIN_ERR_INVALID_ARG;
+    const bool y32 = (flags & kFlagYFp32) != 0;
+    if (!aligned(d_h, 2) || !aligned(d_gamma, 2) || !aligned(d_x_out, 2) || !aligned(d_y, y32 ? 4 : 2))
+        return FLUXBIN_ERR_MISALIGNED;
+    if (d_x_out) {
+        // the kernel reads all of h while writing x: they must not overlap
+        const uintptr_t h0 = reinterpret_cast<uintptr_t>(d_h), x0 = reinterpret_cast<uintptr_t>(d_x_out);
+        const uintptr_t n = (uintptr_t)d.N * 2u;
+        if (x0 < h0 + n && h0 < x0 + n) return FLUXBIN_ERR_INVALID_ARG;
+    }
+    BranchIn g{d_words, d_r, d_c, nullptr, d.N, d.Kb, d.row_scale_group};
+    BranchIn s{d_swords, d_rs, d_cs, d_idx, has_salient(d) ? d.n_sal : 0, d.Ks ? d.Ks : 1, d.sal_scale_group};
+    const BranchIn* brs[2] = {&g, has_salient(d) ? &s : nullptr};
+    for (int q = 0; q < 2; ++q) {
+        const BranchIn* b = brs[q];
+        if (!b || b->ncols == 0) continue;
+        if (!b->words || !b->r || !b->c) return FLUXBIN_ERR_INVALID_ARG;
+        if (!aligned(b->words, 16)) return FLUXBIN_ERR_MISALIGNED;
+        if (!aligned(b->r, 2) || !aligned(b->c, 2) || !aligned(b->gather, 4)) return FLUXBIN_ERR_MISALIGNED;
+    }
+    const int nb1 = has_salient(d) ? d.Ks : 0;
+    if (!d_workspace || workspace_bytes < workspace_bytes_for(d.M, 1) + table_bytes_for(layer_units(d)))
+        return FLUXBIN_ERR_WORKSPACE;
+    if (!aligned(d_workspace, 16)) return FLUXBIN_ERR_MISALIGNED;
+    const NormArgs norm{reinterpret_cast<const __half*>(d_gamma), eps, reinterpret_cast<__half*>(d_x_out)};
+    return run_lut1h(d.M, d.N, g, has_salient(d) ? &s : nullptr, nb1, d_h, d_y, flags, d_workspace, stream, nullptr,
+                     &norm);
 }
 
 }  // extern "C"

@@ -6,7 +6,7 @@
 namespace fluxbin {
 
 using KernelFn = void (*)(KernelArgs);
-using TabKernelFn = void (*)(KernelArgs, float*);
+using TabKernelFn = void (*)(KernelArgs, float*, NormArgs);
 using HKernelFn = void (*)(KernelArgs, const float*);
 
 namespace {
@@ -30,14 +30,16 @@ HKernelFn pick_h(int nb0, int nb1) {
 }
 }  // namespace
 
-TabKernelFn select_tables_kernel(int nb0, int nb1) {
-#define FB_T_NB1(NB0)                                          \
-    switch (nb1) {                                             \
-        case 0: return &fluxbin_tables_kernel<NB0, 0>;        \
-        case 1: return &fluxbin_tables_kernel<NB0, 1>;        \
-        case 2: return &fluxbin_tables_kernel<NB0, 2>;        \
-        case 4: return &fluxbin_tables_kernel<NB0, 4>;        \
-        default: return nullptr;                               \
+namespace {
+template <bool NORM>
+TabKernelFn pick_t(int nb0, int nb1) {
+#define FB_T_NB1(NB0)                                                \
+    switch (nb1) {                                                   \
+        case 0: return &fluxbin_tables_kernel<NB0, 0, NORM>;        \
+        case 1: return &fluxbin_tables_kernel<NB0, 1, NORM>;        \
+        case 2: return &fluxbin_tables_kernel<NB0, 2, NORM>;        \
+        case 4: return &fluxbin_tables_kernel<NB0, 4, NORM>;        \
+        default: return nullptr;                                     \
     }
     switch (nb0) {
         case 1: FB_T_NB1(1)
@@ -46,6 +48,12 @@ TabKernelFn select_tables_kernel(int nb0, int nb1) {
         default: return nullptr;
     }
 #undef FB_T_NB1
+}
+}  // namespace
+
+// norm: the variant fused with the preceding RMS normalisation
+TabKernelFn select_tables_kernel(int nb0, int nb1, bool norm) {
+    return norm ? pick_t<true>(nb0, nb1) : pick_t<false>(nb0, nb1);
 }
 
 HKernelFn select_kernel_lut1h(int spw, int nb0, int nb1) {

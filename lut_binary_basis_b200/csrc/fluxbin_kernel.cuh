@@ -83,6 +83,14 @@ struct KernelArgs {
     unsigned int* err;      // device error word (kernels with bounded waits set a bit when one gives up)
 };
 
+// The element-wise operator preceding a layer, fused into its table
+// precompute (fluxbin_tables.cuh, NORM): RMS normalisation.
+struct NormArgs {
+    const __half* gamma;    // [N] RMSNorm weight
+    float eps;              // added to mean(h^2)
+    __half* x_out;          // [N] normalised activation (fp16), or null
+};
+
 constexpr uint32_t kFlagAccumulate = 1u;
 constexpr uint32_t kFlagYFp32 = 2u;
 constexpr uint32_t kFlagEarlyWeights = 4u;

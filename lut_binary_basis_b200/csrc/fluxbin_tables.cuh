@@ -21,6 +21,15 @@
 // 2v + t/128, the 16 entries of pattern block (t%128)/8 of the four tables in
 // banks 4*(t%8) .. 4*(t%8)+3 in Gray-code order (two paired fp32 adds and one
 // 16-byte store per step).
+//
+// NORM: the precompute fused with the element-wise operator that precedes
+// the layer (LUT Tensor Core notes, Section 3.1.1, fusion of the precompute
+// into the preceding operator), taken to be the RMS normalisation of a
+// LLaMA-style block: the kernel reads the un-normalised activation h and
+// forms x = h (.) gamma / sqrt(mean(h^2) + eps) itself (in fp32, never
+// rounded to fp16 on the way to the tables).  Every CTA sums h^2 over the
+// whole row in the same order, so all of them use the same 1/rms; CTA v also
+// writes its slice of x (rounded to fp16) when asked to.
 #pragma once
 
 #include "fluxbin_kernel.cuh"
@@ -34,9 +43,11 @@ __device__ __forceinline__ void stg_v4(float* p, uint64_t lo, uint64_t hi) {
     asm volatile("st.global.v2.b64 [%0], {%1, %2};" ::"l"(p), "l"(lo), "l"(hi) : "memory");
 }
 
-template <int NB0, int NB1>
-__global__ void __launch_bounds__(kTabThreads) fluxbin_tables_kernel(const KernelArgs a, float* tables) {
+template <int NB0, int NB1, bool NORM>
+__global__ void __launch_bounds__(kTabThreads) fluxbin_tables_kernel(const KernelArgs a, float* tables,
+                                                                      const NormArgs nrm) {
     __shared__ __align__(16) float vbuf[2][8][32];   // [unit of the pair][bit t][bank]
+    __shared__ float wsum[kTabThreads / 32];
     const int tid = threadIdx.x;
     const int U = a.br[0].units + (NB1 > 0 ? a.br[1].units : 0);
     const int v = blockIdx.x;
@@ -52,12 +63,53 @@ __global__ void __launch_bounds__(kTabThreads) fluxbin_tables_kernel(const Kerne
     // x was written by the preceding kernel; the table buffer may still be
     // read by it
     asm volatile("griddepcontrol.wait;" ::: "memory");
+    float r_inv = 1.f;
+    if constexpr (NORM) {
+        // 1/rms of the whole row: per-thread strided sums, then the warps'
+        // sums in warp order (the same order in every CTA)
+        float ss = 0.f;
+        if ((a.N & 7) == 0 && (reinterpret_cast<uintptr_t>(a.x) & 15) == 0) {
+            // 16-byte loads of 8 entries
+            const uint4* h8 = reinterpret_cast<const uint4*>(a.x);
+            for (int n = tid; n < a.N / 8; n += kTabThreads) {
+                const uint4 w = __ldg(h8 + n);
+                const uint32_t q[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&q[e]));
+                    ss = fmaf(f.x, f.x, ss);
+                    ss = fmaf(f.y, f.y, ss);
+                }
+            }
+        } else {
+            for (int n = tid; n < a.N; n += kTabThreads) {
+                const float h = __half2float(a.x[n]);
+                ss = fmaf(h, h, ss);
+            }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+        if (tid % 32 == 0) wsum[tid / 32] = ss;
+        __syncthreads();
+        float tot = 0.f;
+#pragma unroll
+        for (int w = 0; w < kTabThreads / 32; ++w) tot += wsum[w];
+        r_inv = rsqrtf(tot / (float)a.N + nrm.eps);
+        if (nrm.x_out) {
+            const int chunk = (a.N + (int)gridDim.x - 1) / (int)gridDim.x;
+            const int n1 = min(a.N, (v + 1) * chunk);
+            for (int n = v * chunk + tid; n < n1; n += kTabThreads)
+                nrm.x_out[n] = __float2half_rn(__half2float(a.x[n]) * __half2float(nrm.gamma[n]) * r_inv);
+        }
+    }
 #pragma unroll
     for (int q = 0; q < 2; ++q) {
         const SlotStatic s = resolve_slot(a, raw[q]);
         __half xv[1];
         slot_x<1>(a, 0, s.col, xv);
-        vbuf[q][tid / 32][tid % 32] = s.c * __half2float(xv[0]);
+        float xf = __half2float(xv[0]);
+        if constexpr (NORM) xf = (s.col >= 0 && s.col < a.N) ? xf * __half2float(nrm.gamma[s.col]) * r_inv : 0.f;
+        vbuf[q][tid / 32][tid % 32] = s.c * xf;
     }
     __syncthreads();
     const int q = tid / 128, it = tid % 128;

@@ -78,12 +78,14 @@ def lib():
             L.fluxbin_lut_gemv.argtypes = [i32, i32, i32, i32, i32, i32, P, P, P, P, P, i32, P, u32, P, sz, P]
             L.fluxbin_linear.argtypes = [P, P, P, P, P, P, P, P, P, i32, P, u32, P, sz, P]
             L.fluxbin_linear_static_scratch.argtypes = [P, P, P, P, P, P, P, P, P, i32, P, u32, P]
+            L.fluxbin_linear_rmsnorm.argtypes = [P, P, P, P, P, P, P, P, P, P, ctypes.c_float, P, P, u32, P, sz, P]
             L.fluxbin_device_status.argtypes = [ctypes.POINTER(u32)]
             L.fluxbin_fit.argtypes = [i32, i32, i32, i32, i32, P, P, P, P, P, P]
             L.fluxbin_fit_hybrid.argtypes = [i32, i32, i32, i32, i32, i32, P, i32, i32, P, P, P, P, P, P, P, P, P]
             for f in ("fluxbin_packed_sizes", "fluxbin_pack", "fluxbin_workspace_bytes",
                       "fluxbin_layer_workspace_bytes", "fluxbin_lut_gemv",
-                      "fluxbin_linear", "fluxbin_linear_static_scratch", "fluxbin_device_status", "fluxbin_fit",
+                      "fluxbin_linear", "fluxbin_linear_static_scratch", "fluxbin_linear_rmsnorm",
+                      "fluxbin_device_status", "fluxbin_fit",
                       "fluxbin_fit_hybrid"):
                 getattr(L, f).restype = ctypes.c_int
             _lib = L
@@ -186,6 +188,20 @@ def fluxbin_linear(desc: LayerDesc, words, r, c, swords, rs, cs, idx, x, B: int,
     _check(lib().fluxbin_linear(ctypes.byref(desc), _dptr(words), _dptr(r), _dptr(c), _dptr(swords), _dptr(rs),
                                 _dptr(cs), _dptr(idx), _dptr(x), B, _dptr(y), flags, _dptr(workspace), wsb,
                                 _stream(stream)), "fluxbin_linear")
+
+
+def fluxbin_linear_rmsnorm(desc: LayerDesc, words, r, c, swords, rs, cs, idx, h, gamma, eps: float, x_out, y,
+                           flags: int = FLAG_Y_FP32, workspace=None, workspace_bytes: Optional[int] = None,
+                           stream=None) -> None:
+    """y (+)= W (h * gamma / sqrt(mean(h^2) + eps)) at batch 1, the table
+    precompute fused with the RMS normalisation (include/fluxbin.h);
+    x_out (fp16 [N] or None) receives the normalised activation."""
+    wsb = workspace_bytes if workspace_bytes is not None else (
+        workspace.numel() * workspace.element_size() if workspace is not None else 0)
+    _check(lib().fluxbin_linear_rmsnorm(ctypes.byref(desc), _dptr(words), _dptr(r), _dptr(c), _dptr(swords),
+                                        _dptr(rs), _dptr(cs), _dptr(idx), _dptr(h), _dptr(gamma), float(eps),
+                                        _dptr(x_out), _dptr(y), flags, _dptr(workspace), wsb, _stream(stream)),
+           "fluxbin_linear_rmsnorm")
 
 
 def fluxbin_linear_static_scratch(desc: LayerDesc, words, r, c, swords, rs, cs, idx, x, B: int, y,
@@ -295,6 +311,11 @@ class DeviceLayer:
         B = x.shape[0] if x.dim() == 2 else 1
         fluxbin_linear(self.desc, self.words, self.r, self.c, self.swords, self.rs, self.cs, self.idx, x, B, y,
                        flags, workspace, None, stream)
+
+    def linear_rmsnorm(self, h, gamma, eps: float, y, flags: int = FLAG_Y_FP32, workspace=None, x_out=None,
+                       stream=None) -> None:
+        fluxbin_linear_rmsnorm(self.desc, self.words, self.r, self.c, self.swords, self.rs, self.cs, self.idx, h,
+                               gamma, eps, x_out, y, flags, workspace, None, stream)
 
 
 def new_workspace(M: int, B: int, device="cuda"):

@@ -53,6 +53,8 @@ def _load():
             lib.oracle_linear_rows.restype = None
             lib.oracle_lut_linear_rows.argtypes = [i64, i64, i32, i32, P, P, P, i32, i64, i32, P, P, P, P,
                                                    i32, i32, i32, i32, P, i64, P, P]
+            lib.oracle_rmsnorm.argtypes = [i64, P, P, ctypes.c_double, P]
+            lib.oracle_rmsnorm.restype = None
             lib.oracle_round_fp16.argtypes = [ctypes.c_double]
             lib.oracle_round_fp16.restype = ctypes.c_double
             lib.oracle_quantize_table_int8.argtypes = [P, i64]
@@ -157,6 +159,23 @@ def gemv_rows(W: np.ndarray, x) -> np.ndarray:
 
 
 TABLE_QUANT = {"none": 0, "fp16": 1, "int8": 2}
+
+
+def rmsnorm(h, gamma, eps: float) -> np.ndarray:
+    """x = h * gamma / sqrt(mean(h^2) + eps) in fp64: the element-wise
+    operator taken to precede a layer whose table precompute is fused into it
+    (one activation row, [N])."""
+    hh = _f64(np.asarray(h).reshape(-1)).copy()
+    gg = _f64(np.asarray(gamma).reshape(-1)).copy()
+    assert hh.size == gg.size and hh.size > 0
+    x = np.zeros(hh.size, np.float64)
+    _load().oracle_rmsnorm(hh.size, _ptr(hh), _ptr(gg), float(eps), _ptr(x))
+    return x
+
+
+def linear_rmsnorm(layer, h, gamma, eps: float) -> np.ndarray:
+    """y = W rmsnorm(h) for one activation row, [1][M]."""
+    return linear(layer, rmsnorm(h, gamma, eps)[None, :])
 
 
 def round_fp16(v: float) -> float:

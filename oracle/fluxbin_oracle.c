@@ -184,6 +184,20 @@ double oracle_lut_lookup_sym(const double* Th, int mu, int64_t p) {
  * significand), from the format's definition: 10 fraction bits, exponents
  * -14 .. 15, subnormal spacing 2^-24, values at or beyond 65520 overflow.
  */
+/*
+ * The element-wise operator taken to precede a layer when the table
+ * precompute is fused into it (LUT Tensor Core notes, Section 3.1.1): the RMS
+ * normalisation of a LLaMA-style block,
+ *     x[n] = h[n] * gamma[n] / sqrt(mean_m(h[m]^2) + eps),
+ * the definition written out in fp64 (no rounding of x).
+ */
+void oracle_rmsnorm(int64_t N, const double* h, const double* gamma, double eps, double* x) {
+    double ss = 0.0;
+    for (int64_t n = 0; n < N; ++n) ss += h[n] * h[n];
+    const double rms = sqrt(ss / (double)N + eps);
+    for (int64_t n = 0; n < N; ++n) x[n] = h[n] * gamma[n] / rms;
+}
+
 double oracle_round_fp16(double v) {
     if (v != v) return v;
     double a = fabs(v);
