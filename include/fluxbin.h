@@ -314,7 +314,7 @@ int fluxbin_linear(const fluxbin_layer_desc* desc,
  * runs on those tables.
  *   d_h       fp16 [N], the un-normalised activation
  *   d_gamma   fp16 [N], the normalisation weight
- *   eps       >= 0, finite
+ *   eps       >= 0, finite (with eps == 0 a row h == 0 divides by zero: x and y are NaN)
  *   d_x_out   fp16 [N] or NULL: if given, receives x rounded to fp16 (round to
  *             nearest even), e.g. for the other layers that read the same x;
  *             must not overlap d_h
