@@ -227,6 +227,31 @@ Plan make_plan(KernelFn fn, int dev, const CtaShape& cs, int64_t Ms, int64_t U, 
     const int64_t ks_wide = (U + units_wide - 1) / units_wide;
     const bool wide_ok = have_ws && ks_wide >= 2;
 
+    // One CTA per SM and more CTA groups than slots: without a split the last
+    // wave runs partly empty.  A split through the workspace that evens the
+    // waves out pays for its reduction; each further split costs ~4% of a
+    // CTA's time (B200, 28672x8192 at batch 16 on the batch-pair kernel:
+    // 224 CTAs 168.7 us, split 2 174.8, 3 154.6, 4 164.4, 6 167.7; the model
+    // ceil(groups*ks/slots)/ks * (1 + 0.04 (ks-1)) ranks them the same way).
+    if (fill_gpu && have_ws && groups > slots && U >= 2) {
+        auto cost = [&](int64_t ks) {
+            return (double)((groups * ks + slots - 1) / slots) / (double)ks * (1.0 + 0.04 * (double)(ks - 1));
+        };
+        const double base = cost(1);
+        int64_t best = 1;
+        double best_cost = base;
+        for (int64_t ks = 2; ks <= std::min<int64_t>(U, 8); ++ks)
+            if (cost(ks) < best_cost) {
+                best = ks;
+                best_cost = cost(ks);
+            }
+        if (best > 1 && best_cost < 0.98 * base) {
+            p.n_ks = (int)best;
+            p.cluster = false;
+            return p;
+        }
+    }
+
     int64_t want = slots / groups;
     if (want > U) want = U;
     if (want > kMaxCluster) want = kMaxCluster;
