@@ -141,8 +141,12 @@ typedef struct fluxbin_layer_desc {
                                          operator) and look them up from shared-memory copies of the
                                          table buffer; needs fluxbin_layer_workspace_bytes() of
                                          workspace (WORKSPACE otherwise), UNSUPPORTED for other
-                                         layers, INVALID_ARG with FLUXBIN_FLAG_PATH_TC.  Measured
-                                         slower than the default on B200 (see the batch-1 kernels). */
+                                         layers, INVALID_ARG with FLUXBIN_FLAG_PATH_TC.  The table
+                                         buffer (the bytes from fluxbin_workspace_bytes(M, 1) on) is
+                                         left holding the tables: only the bytes before it are left
+                                         zero-filled, so a workspace shared with other calls must not
+                                         put that buffer where they need zeros.  Measured slower
+                                         than the default on B200 (see the batch-1 kernels). */
 #define FLUXBIN_FLAG_TEST_WAIT_TIMEOUT 32u /* test hook, only together with FLUXBIN_FLAG_PATH_TC: the
                                          tensor-core kernel's preparing warps never report a buffer
                                          ready and every wait gives up after a few polls, so the
@@ -321,7 +325,8 @@ int fluxbin_linear(const fluxbin_layer_desc* desc,
  *   flags     FLUXBIN_FLAG_ACCUMULATE, FLUXBIN_FLAG_Y_FP32,
  *             FLUXBIN_FLAG_EARLY_WEIGHTS only
  *   d_workspace, workspace_bytes   at least fluxbin_layer_workspace_bytes(desc, 1)
- *             (the split-K scratch plus the table buffer), 16-byte aligned
+ *             (the split-K scratch plus the table buffer), 16-byte aligned; as with
+ *             FLUXBIN_FLAG_SEPARATE_TABLES the table buffer is left holding the tables
  * Other arguments as for fluxbin_linear.  Layers: mu = 8 with per-row scales
  * in both branches (else UNSUPPORTED).  M == 0 returns FLUXBIN_OK without
  * launching (x_out is then not written); N == 0 with M > 0 is BAD_SHAPE.
