@@ -2,6 +2,7 @@
 // selection, grid sizing and the launch.  Declarations and the full contract
 // are in include/fluxbin.h.
 #include <algorithm>
+#include <cmath>
 #include <cuda_runtime.h>
 
 #include <cstdio>
@@ -588,8 +589,8 @@ int run_lut2(int32_t M, int32_t N, const BranchIn& g, const BranchIn* s, int nb1
 
 // Batch 1, mu = 8, per-row scales, with room for the table buffer in the
 // workspace: the table precompute as its own kernel (fluxbin_tables.cuh),
-// then the lookups on the precomputed tables (fluxbin_lut1h.cuh).  2048 rows
-// per CTA when that plan keeps most SMs busy, else 1024.
+// then the lookups on the precomputed tables (fluxbin_lut1h.cuh), 1024 or
+// 2048 rows per CTA.
 int run_lut1h(int32_t M, int32_t N, const BranchIn& g, const BranchIn* s, int nb1, const uint16_t* d_x, void* d_y,
               uint32_t flags, void* ws, void* stream, int* uses_ws, const NormArgs* norm = nullptr) {
     int dev = 0;
@@ -618,7 +619,12 @@ int run_lut1h(int32_t M, int32_t N, const BranchIn& g, const BranchIn* s, int nb
         if ((st = func_info_shape(k2, dev, c2.smem, c2.threads, di, &i2)) != FLUXBIN_OK) return st;
         const Plan p4 = make_plan(k4, dev, c4, a.Ms, U, 1, di, i4, true, true);
         const Plan p2 = make_plan(k2, dev, c2, a.Ms, U, 1, di, i2, true, true);
-        if ((int64_t)p4.n_rg * p4.n_ks * 4 >= (int64_t)di.sm_count * 3) {
+        // 1024 rows per CTA whenever that plan keeps three quarters of the
+        // SMs busy (the 2048-row build spills; B200, batch 1: 28672x8192
+        // 28.5 -> 27.1 us, 8192x28672 30.9 -> 29.0 us), else 2048 if that
+        // one does
+        const auto fills = [&](const Plan& p) { return (int64_t)p.n_rg * p.n_ks * 4 >= (int64_t)di.sm_count * 3; };
+        if (!fills(p2) && fills(p4)) {
             fn = f4;
             plan = p4;
         } else {
@@ -935,7 +941,7 @@ int fluxbin_linear_rmsnorm(const fluxbin_layer_desc* desc, const uint32_t* d_wor
     if (st != FLUXBIN_OK) return st;
     const fluxbin_layer_desc& d = *desc;
     if (flags & ~(kFlagAccumulate | kFlagYFp32 | kFlagEarlyWeights)) return FLUXBIN_ERR_INVALID_ARG;
-    if (!(eps >= 0.f) || eps > 3.0e38f) return FLUXBIN_ERR_INVALID_ARG;   // negative, NaN or infinite
+    if (!(eps >= 0.f) || !std::isfinite(eps)) return FLUXBIN_ERR_INVALID_ARG;   // negative, NaN or infinite
     if (d.M == 0) return FLUXBIN_OK;
     if (d.N == 0) return FLUXBIN_ERR_BAD_SHAPE;   // no mean of h^2 to take
     if (!hoistable(d, 1)) return FLUXBIN_ERR_UNSUPPORTED;
