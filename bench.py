@@ -915,6 +915,9 @@ def main(argv=None):
                     help="time the host decomposition fitter (library vs oracle) on a dense matrix instead")
     ap.add_argument("--fit-size", type=int, default=4096)
     ap.add_argument("--fit-iters", type=int, default=5)
+    ap.add_argument("--fusion", action="store_true",
+                    help="time the headline layer with its table precompute fused into the preceding RMS "
+                         "normalisation, against the precompute on a normalised row and the default path, instead")
     args = ap.parse_args(argv)
     args.warmup = max(3, args.warmup)
     rank, local_rank, world = dist_env()
@@ -926,6 +929,17 @@ def main(argv=None):
         return
     if args.fit:
         print(json.dumps(run_fit(args)), flush=True)
+        return
+    if args.fusion:
+        import torch
+        import __graft_entry__
+        from lut_binary_basis_b200 import synth
+        __graft_entry__.build()
+        device = torch.device("cuda", 0)
+        torch.cuda.set_device(device)
+        sp = headline_spec()
+        layer = synth.make_layer(sp, synth.layer_key(HEADLINE_WID, 0, 0))
+        print(json.dumps(precompute_fusion_entry(sp, layer, device, HEADLINE_WID, steps=args.steps)), flush=True)
         return
     if args.impl == "reference":
         res = run_reference(args, rank, world)
