@@ -663,8 +663,8 @@ int run_lut1h(int32_t M, int32_t N, const BranchIn& g, const BranchIn* s, int nb
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cudaLaunchConfig_t tc = {};
-    tc.gridDim = dim3((unsigned)((U + 1) / 2));
-    tc.blockDim = dim3(256);   // fluxbin_tables_kernel: one unit pair per CTA of 256 threads
+    tc.gridDim = dim3((unsigned)U);
+    tc.blockDim = dim3(256);   // fluxbin_tables_kernel: one unit per CTA of 256 threads
     tc.stream = static_cast<cudaStream_t>(stream);
     tc.attrs = attr;
     tc.numAttrs = 1;

@@ -16,11 +16,11 @@
 // which is exactly the shared-memory layout the lookups address (one 64 KiB
 // copy per unit pair).  The bank of table (base k, sub-vector j) is k*P + j.
 //
-// One CTA of 256 threads builds one unit pair: the 512 activation products
-// (two per thread) go to shared memory, then thread t builds, for unit
-// 2v + t/128, the 16 entries of pattern block (t%128)/8 of the four tables in
-// banks 4*(t%8) .. 4*(t%8)+3 in Gray-code order (two paired fp32 adds and one
-// 16-byte store per step).
+// One CTA of 256 threads builds one unit: the 256 activation products (one
+// per thread) go to shared memory, then thread t builds the 8 entries
+// (hi << 4) | (half << 3) | 0..7 of the four tables in banks 4 qd .. 4 qd + 3
+// (t/2 = 8 hi + qd, half = t % 2) in Gray-code order (two paired fp32 adds
+// and one 16-byte store per step).
 //
 // NORM: the precompute fused with the element-wise operator that precedes
 // the layer (LUT Tensor Core notes, Section 3.1.1, fusion of the precompute
@@ -46,20 +46,14 @@ __device__ __forceinline__ void stg_v4(float* p, uint64_t lo, uint64_t hi) {
 template <int NB0, int NB1, bool NORM>
 __global__ void __launch_bounds__(kTabThreads) fluxbin_tables_kernel(const KernelArgs a, float* tables,
                                                                       const NormArgs nrm) {
-    __shared__ __align__(16) float vbuf[2][8][32];   // [unit of the pair][bit t][bank]
+    __shared__ __align__(16) float vbuf[8][32];   // [bit t][bank]
     __shared__ float wsum[kTabThreads / 32];
     const int tid = threadIdx.x;
-    const int U = a.br[0].units + (NB1 > 0 ? a.br[1].units : 0);
-    const int v = blockIdx.x;
+    const int u = blockIdx.x;              // one unit per CTA
+    const int v = u >> 1, h = u & 1;       // its pair and half in the table buffer
     asm volatile("griddepcontrol.launch_dependents;");
-    // layer data of this thread's two product slots (before the dependency wait)
-    SlotRaw raw[2];
-#pragma unroll
-    for (int q = 0; q < 2; ++q) {
-        const int u = 2 * v + q;
-        raw[q] = SlotRaw{__float2half(0.f), -1};
-        if (u < U) raw[q] = slot_raw<8, NB0, NB1>(a, u, tid);
-    }
+    // layer data of this thread's product slot (before the dependency wait)
+    const SlotRaw raw = slot_raw<8, NB0, NB1>(a, u, tid);
     // x was written by the preceding kernel; the table buffer may still be
     // read by it
     asm volatile("griddepcontrol.wait;" ::: "memory");
@@ -73,18 +67,18 @@ __global__ void __launch_bounds__(kTabThreads) fluxbin_tables_kernel(const Kerne
             const uint4* h8 = reinterpret_cast<const uint4*>(a.x);
             for (int n = tid; n < a.N / 8; n += kTabThreads) {
                 const uint4 w = __ldg(h8 + n);
-                const uint32_t q[4] = {w.x, w.y, w.z, w.w};
+                const uint32_t qw[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
-                    const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&q[e]));
+                    const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&qw[e]));
                     ss = fmaf(f.x, f.x, ss);
                     ss = fmaf(f.y, f.y, ss);
                 }
             }
         } else {
             for (int n = tid; n < a.N; n += kTabThreads) {
-                const float h = __half2float(a.x[n]);
-                ss = fmaf(h, h, ss);
+                const float hv = __half2float(a.x[n]);
+                ss = fmaf(hv, hv, ss);
             }
         }
 #pragma unroll
@@ -97,47 +91,48 @@ __global__ void __launch_bounds__(kTabThreads) fluxbin_tables_kernel(const Kerne
         r_inv = rsqrtf(tot / (float)a.N + nrm.eps);
         if (nrm.x_out) {
             const int chunk = (a.N + (int)gridDim.x - 1) / (int)gridDim.x;
-            const int n1 = min(a.N, (v + 1) * chunk);
-            for (int n = v * chunk + tid; n < n1; n += kTabThreads)
+            const int n1 = min(a.N, (u + 1) * chunk);
+            for (int n = u * chunk + tid; n < n1; n += kTabThreads)
                 nrm.x_out[n] = __float2half_rn(__half2float(a.x[n]) * __half2float(nrm.gamma[n]) * r_inv);
         }
     }
-#pragma unroll
-    for (int q = 0; q < 2; ++q) {
-        const SlotStatic s = resolve_slot(a, raw[q]);
+    {
+        const SlotStatic sl = resolve_slot(a, raw);
         __half xv[1];
-        slot_x<1>(a, 0, s.col, xv);
+        slot_x<1>(a, 0, sl.col, xv);
         float xf = __half2float(xv[0]);
-        if constexpr (NORM) xf = (s.col >= 0 && s.col < a.N) ? xf * __half2float(nrm.gamma[s.col]) * r_inv : 0.f;
-        vbuf[q][tid / 32][tid % 32] = s.c * xf;
+        if constexpr (NORM) xf = (sl.col >= 0 && sl.col < a.N) ? xf * __half2float(nrm.gamma[sl.col]) * r_inv : 0.f;
+        vbuf[tid / 32][tid % 32] = sl.c * xf;
     }
     __syncthreads();
-    const int q = tid / 128, it = tid % 128;
-    if (2 * v + q >= U) return;
+    // thread t: entries (hi << 4) | (half << 3) | 0..7 of the four tables in
+    // banks 4 qd .. 4 qd + 3, with it = t/2 = 8 hi + qd and half = t % 2
+    const int it = tid >> 1, half = tid & 1;
     const int hi = it / 8, qd = it % 8;
     constexpr uint64_t kSign2 = 0x8000000080000000ull;
-    uint64_t T0 = 0, T1 = 0, d0[4], d1[4];
+    uint64_t T0 = 0, T1 = 0, d0[3], d1[3];
 #pragma unroll
-    for (int t = 4; t < 8; ++t) {
-        const uint64_t flip = ((hi >> (t - 4)) & 1) ? 0ull : kSign2;
-        const uint64_t v0 = *reinterpret_cast<const uint64_t*>(&vbuf[q][t][4 * qd]) ^ flip;
-        const uint64_t v1 = *reinterpret_cast<const uint64_t*>(&vbuf[q][t][4 * qd + 2]) ^ flip;
-        T0 = t == 4 ? v0 : add_f32x2(T0, v0);
-        T1 = t == 4 ? v1 : add_f32x2(T1, v1);
+    for (int t = 3; t < 8; ++t) {
+        const bool plus = t == 3 ? half != 0 : ((hi >> (t - 4)) & 1) != 0;
+        const uint64_t flip = plus ? 0ull : kSign2;
+        const uint64_t v0 = *reinterpret_cast<const uint64_t*>(&vbuf[t][4 * qd]) ^ flip;
+        const uint64_t v1 = *reinterpret_cast<const uint64_t*>(&vbuf[t][4 * qd + 2]) ^ flip;
+        T0 = t == 3 ? v0 : add_f32x2(T0, v0);
+        T1 = t == 3 ? v1 : add_f32x2(T1, v1);
     }
 #pragma unroll
-    for (int t = 0; t < 4; ++t) {
-        const uint64_t v0 = *reinterpret_cast<const uint64_t*>(&vbuf[q][t][4 * qd]);
-        const uint64_t v1 = *reinterpret_cast<const uint64_t*>(&vbuf[q][t][4 * qd + 2]);
+    for (int t = 0; t < 3; ++t) {
+        const uint64_t v0 = *reinterpret_cast<const uint64_t*>(&vbuf[t][4 * qd]);
+        const uint64_t v1 = *reinterpret_cast<const uint64_t*>(&vbuf[t][4 * qd + 2]);
         T0 = sub_f32x2(T0, v0);
         T1 = sub_f32x2(T1, v1);
         d0[t] = add_f32x2(v0, v0);
         d1[t] = add_f32x2(v1, v1);
     }
-    // entry e of bank 4 qd at float index v*16384 + e*64 + q*32 + 4 qd
-    float* base = tables + (int64_t)v * (kTabPairBytes / 4) + (hi << 4) * 64 + q * 32 + 4 * qd;
+    // entry e of bank 4 qd at float index v*16384 + e*64 + h*32 + 4 qd
+    float* base = tables + (int64_t)v * (kTabPairBytes / 4) + ((hi << 4) | (half << 3)) * 64 + h * 32 + 4 * qd;
     stg_v4(base, T0, T1);
-    static_for<1, 16>([&](auto ic) {
+    static_for<1, 8>([&](auto ic) {
         constexpr int i = decltype(ic)::value;
         constexpr int t = lowest_bit(i);
         constexpr int g = i ^ (i >> 1);
